@@ -1,0 +1,494 @@
+"""Benchmark of the weight-only skinny GEMM on B200.
+
+One step = one decoder layer's weight-only GEMMs (three 5120x5120 NVFP4
+attention projections, the 34816x5120 NVFP4 gate+up and the 5120x17408 FP8
+down projection) at M = 1 (one decode token) and then at M = 8 (a k=7
+speculative-verify round plus its base token): ten kernel launches.  Weights
+rotate through three device copies (702 MB, over 5x the 126 MB L2), so no
+launch finds its weights in L2.
+
+Metric: effective HBM GB/s = (packed weight bytes + scale bytes + activation
+bytes + output bytes) / device time, with the fraction of the measured HBM
+copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(replicas: the GEMMs of different requests shard with no exchange); rank 0
+prints one JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic_inputs as si  # noqa: E402
+
+METRIC = "NVFP4/FP8 skinny-GEMM effective HBM GB/s & % of B200 peak at M=1 and M=8"
+WORKLOAD = "decoder_layer_m1_m8"
+PASSES = (1, 8)          # M of the two passes of a step
+COPIES = 3               # weight copies in rotation
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ("skinny.cu", "ptx.cuh", "layout.h")
+
+
+# ---------------------------------------------------------------------------
+# Byte accounting (algorithmic bytes: what the operation must move at least)
+# ---------------------------------------------------------------------------
+
+def out_bytes(spec) -> int:
+    return 4 if spec.out == "f32" else 2
+
+
+def weight_bytes(spec) -> int:
+    if spec.fmt == "nvfp4":
+        return spec.N * spec.K // 2 + spec.N * spec.K // 16 + 4
+    return spec.N * spec.K + 4 * spec.N
+
+
+def gemm_bytes(spec, M: int) -> int:
+    return weight_bytes(spec) + M * spec.K * 2 + M * spec.N * out_bytes(spec)
+
+
+def step_bytes() -> int:
+    return sum(gemm_bytes(s, M) for M in PASSES for s in si.MIXED_LAYER)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "fp8_weight_only_w4a16_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(avg_alg_bytes: float):
+    """DRAM bytes per launch of the NVFP4 kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "nvfp4_gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_sha") != kernel_source_hash():
+        return None
+    return float(d["dram_bytes_per_alg_byte"]) * avg_alg_bytes
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), "--query-gpu=timestamp," + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Workload on the device
+# ---------------------------------------------------------------------------
+
+def build_device_workload(dev):
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    weights = [[] for _ in range(COPIES)]
+    for i, spec in enumerate(si.MIXED_LAYER):
+        logical = si.weights_for(spec, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=10 * i)
+        if spec.fmt == "nvfp4":
+            pc, ps = sk.pack_nvfp4(*logical)
+            base = (torch.from_numpy(pc).to(dev), torch.from_numpy(ps).to(dev))
+            for c in range(COPIES):
+                cc, cs = (base[0], base[1]) if c == 0 else (base[0].clone(), base[1].clone())
+                weights[c].append(sk.PackedNVFP4(cc, cs, spec.global_scale, spec.N, spec.K))
+        else:
+            pc = torch.from_numpy(sk.pack_fp8(logical[0])).to(dev)
+            s = torch.from_numpy(logical[1]).to(dev)
+            for c in range(COPIES):
+                weights[c].append(sk.PackedFP8(pc if c == 0 else pc.clone(), s if c == 0 else s.clone(),
+                                               spec.N, spec.K))
+    xs = {M: [torch.from_numpy(si.activations(M, spec.K, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=100 + i)).to(dev)
+              for i, spec in enumerate(si.MIXED_LAYER)] for M in PASSES}
+    ys = {M: [torch.empty((M, spec.N), dtype=torch.float32 if spec.out == "f32" else torch.float16, device=dev)
+              for spec in si.MIXED_LAYER] for M in PASSES}
+    need = max(sk.workspace_bytes(w.fmt, M, w.N, w.K) for w in weights[0] for M in PASSES)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    return weights, xs, ys, ws
+
+
+def copy_for(step: int, pass_idx: int) -> int:
+    return (2 * step + pass_idx) % COPIES
+
+
+def launch_step(weights, xs, ys, ws, step: int, events=None):
+    """Enqueue one step (both passes) on the current stream; optionally record an
+    event before each launch and after the last one."""
+    import fp8_weight_only_w4a16_b200 as sk
+
+    k = 0
+    for pi, M in enumerate(PASSES):
+        wc = weights[copy_for(step, pi)]
+        for i in range(len(si.MIXED_LAYER)):
+            if events is not None:
+                events[k].record()
+            sk.gemm_into(ys[M][i], xs[M][i], wc[i], workspace=ws)
+            k += 1
+    if events is not None:
+        events[k].record()
+
+
+def capture_step_graphs(weights, xs, ys, ws, with_events: bool):
+    """One CUDA graph per rotation phase (a step's launches are fixed by step % 3)."""
+    import torch
+
+    graphs, evsets = [], []
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        launch_step(weights, xs, ys, ws, 0)  # warm the driver paths before capture
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    for phase in range(COPIES):
+        evs = [torch.cuda.Event(enable_timing=True, external=True)
+               for _ in range(len(PASSES) * len(si.MIXED_LAYER) + 1)] if with_events else None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            launch_step(weights, xs, ys, ws, phase, evs)
+        graphs.append(g)
+        evsets.append(evs)
+    return graphs, evsets
+
+
+def per_kernel_durations(graphs, evsets, rounds: int):
+    """Replay the event-instrumented step graphs; returns ms per launch [pass][gemm] (mean)."""
+    import torch
+
+    nl = len(si.MIXED_LAYER)
+    acc = np.zeros((len(PASSES), nl))
+    cnt = 0
+    for r in range(rounds):
+        for phase in range(COPIES):
+            graphs[phase].replay()
+            torch.cuda.synchronize()
+            evs = evsets[phase]
+            for k in range(len(PASSES) * nl):
+                acc[k // nl, k % nl] += evs[k].elapsed_time(evs[k + 1])
+            cnt += 1
+    return acc / cnt
+
+
+def e2e_run(weights, xs, ys, ws, steps: int, warmup: int):
+    """Same workload through the public API with host buffers: every step copies
+    its activations from pinned host memory and reads every output back."""
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    hx = {M: [x.cpu().pin_memory() for x in xs[M]] for M in PASSES}
+    hy = {M: [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys[M]] for M in PASSES}
+    h2d = sum(x.numel() * x.element_size() for M in PASSES for x in hx[M])
+    d2h = sum(y.numel() * y.element_size() for M in PASSES for y in hy[M])
+
+    def one(step):
+        for pi, M in enumerate(PASSES):
+            wc = weights[copy_for(step, pi)]
+            for i in range(len(si.MIXED_LAYER)):
+                xs[M][i].copy_(hx[M][i], non_blocking=True)
+                sk.gemm_into(ys[M][i], xs[M][i], wc[i], workspace=ws)
+                hy[M][i].copy_(ys[M][i], non_blocking=True)
+
+    graphs = []
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        one(0)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    for phase in range(COPIES):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one(phase)
+        graphs.append(g)
+    for i in range(warmup):
+        graphs[i % COPIES].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        graphs[i % COPIES].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# The oracle on the host cores (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_inputs(frac: float):
+    """Row samples of every GEMM of a step (both passes), as oracle inputs."""
+    items = []
+    for i, spec in enumerate(si.MIXED_LAYER):
+        rows = max(1, int(round(spec.N * frac)))
+        sub = si.GemmSpec(spec.name, spec.fmt, rows, spec.K, spec.scale_dist, spec.global_scale, spec.out)
+        logical = si.weights_for(sub, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=10 * i)
+        for M in PASSES:
+            x = si.activations(M, spec.K, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=100 + i)
+            items.append((sub, M, logical, x))
+    return items
+
+
+def _oracle_run(items, threads):
+    import oracle
+
+    t0 = time.perf_counter()
+    for spec, M, logical, x in items:
+        if spec.fmt == "nvfp4":
+            oracle.nvfp4_gemm(x, logical[0], logical[1], spec.global_scale, threads=threads)
+        else:
+            oracle.fp8_gemm(x, logical[0], logical[1], threads=threads)
+    return time.perf_counter() - t0
+
+
+def _oracle_bytes(items) -> int:
+    return sum(gemm_bytes(spec, M) for spec, M, _, _ in items)
+
+
+def oracle_sample_frac(target_s: float, threads: int) -> float:
+    probe = 1.0 / 2048
+    t = _oracle_run(_oracle_inputs(probe), threads)
+    frac = probe * target_s / max(t, 1e-3)
+    return float(min(1.0, max(probe, frac)))
+
+
+def cpu_baseline(target_s: float = 12.0):
+    import oracle
+
+    threads = oracle.default_threads()
+    frac = oracle_sample_frac(target_s, threads)
+    items = _oracle_inputs(frac)
+    t = _oracle_run(items, threads)
+    return {"value": round(_oracle_bytes(items) / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "float64 C oracle, %d threads, on the first %.3f%% of the rows of each of the 5 GEMMs of %s at "
+                      "M=1 and M=8 (same byte formula), %.1f s" % (threads, 100 * frac, WORKLOAD, t)}
+
+
+def reference_arm(args):
+    """The oracle as the reference arm: each step a bounded row sample of the workload."""
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    threads = oracle.default_threads()
+    per_step_s = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    frac = oracle_sample_frac(per_step_s, threads)
+    items = _oracle_inputs(frac)
+    for _ in range(args.warmup):
+        _oracle_run(items, threads)
+    t = sum(_oracle_run(items, threads) for _ in range(args.steps))
+    value = _oracle_bytes(items) * args.steps / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample_rows_frac": frac},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": "float64 C oracle on the first %.3f%% of the rows of each GEMM of %s "
+                                       "at M=1 and M=8" % (100 * frac, WORKLOAD)},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Main (our arm)
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="skinny", choices=["skinny", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--event-rounds", type=int, default=20)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    peak, peak_src = load_peaks()
+    weights, xs, ys, ws = build_device_workload(dev)
+    graphs, _ = capture_step_graphs(weights, xs, ys, ws, with_events=False)
+    egraphs, evsets = capture_step_graphs(weights, xs, ys, ws, with_events=True)
+
+    sampler = ClockSampler(local)
+    # Per-launch durations (CUDA events on the launching stream, inside the
+    # replayed graphs) -- this also brings the GPU to its loaded clocks.
+    dur = per_kernel_durations(egraphs, evsets, args.event_rounds)
+
+    for i in range(args.warmup):
+        graphs[i % COPIES].replay()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % COPIES].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert sk.device_error(clear=True) == 0, "a device-side wait gave up"
+
+    e2e_ms, h2d, d2h = e2e_run(weights, xs, ys, ws, args.steps, args.warmup)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    sb = step_bytes()
+    value = world * sb * args.steps / (ms * 1e-3) / 1e9
+    e2e_value = world * sb * args.steps / (e2e_ms * 1e-3) / 1e9
+
+    # Roofline of the dominant kernel (the NVFP4 GEMM: 8 of 10 launches, most of the bytes).
+    per = []
+    nv_bytes = nv_ms = 0.0
+    nv_launches = 0
+    for pi, M in enumerate(PASSES):
+        for i, spec in enumerate(si.MIXED_LAYER):
+            b = gemm_bytes(spec, M)
+            d = float(dur[pi, i])
+            per.append({"gemm": spec.name, "fmt": spec.fmt, "M": M, "N": spec.N, "K": spec.K,
+                        "us": round(1e3 * d, 3), "GB/s": round(b / (d * 1e-3) / 1e9, 1),
+                        "frac": round(b / (d * 1e-3) / 1e9 / peak, 4)})
+            if spec.fmt == "nvfp4":
+                nv_bytes += b
+                nv_ms += d
+                nv_launches += 1
+    achieved = nv_bytes / (nv_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(nv_bytes / nv_launches)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD,
+                   "gemms": ["%s %s %dx%d" % (s.name, s.fmt, s.N, s.K) for s in si.MIXED_LAYER],
+                   "M": list(PASSES), "operands": "NVFP4/FP8 weights x FP16 activations, FP32 accumulation",
+                   "l2": "inputs larger than L2: %d rotating weight copies, %.0f MB" %
+                         (COPIES, COPIES * sum(weight_bytes(s) for s in si.MIXED_LAYER) / 1e6),
+                   "bytes_per_step": sb, "launch": "CUDA graph per step", "parallelism": "replicas" if world > 1
+                   else "single GPU"},
+        "frac_of_peak": round(value / world / peak, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                     "kernel": "gemm_kernel<NVFP4>", "launches_timed": nv_launches * args.event_rounds * COPIES},
+        "per_gemm": per,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(PASSES) * len(si.MIXED_LAYER) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    del graphs, egraphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

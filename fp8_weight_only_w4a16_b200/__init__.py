@@ -1,0 +1,262 @@
+"""B200-native weight-only skinny GEMM: y[M,N] = x[M,K] . W^T, M = 1..8,
+with W kept in HBM as NVFP4 (E2M1 codes + UE4M3 per-16 scales + FP32 global)
+or FP8 E4M3 (+ FP32 per output channel), FP16 activations, FP32 accumulation.
+
+This module is a thin ctypes binding over ``libskinny.so`` (whose C ABI is
+``include/skinny.h``): it turns numpy arrays and torch tensors into pointers,
+sizes and a stream handle, calls the library, and raises ``SkinnyError`` on a
+non-zero status.  Every step of the GEMM runs in the library's CUDA kernels;
+there is no fallback: if the library is missing, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "libskinny.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_ALIGNMENT = -3
+ERR_CUDA = -4
+ERR_WORKSPACE = -5
+
+OUT_F16 = 0
+OUT_F32 = 1
+FMT_NVFP4 = 0
+FMT_FP8 = 1
+MAX_M = 8
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SkinnyError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (%d)" % (what, status_string(status), status))
+
+
+def library() -> ctypes.CDLL:
+    """Load libskinny.so (built by ``__graft_entry__.build()``); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIBRARY_PATH):
+                raise RuntimeError("libskinny.so is not built (%s); run __graft_entry__.build()" % LIBRARY_PATH)
+            lib = ctypes.CDLL(LIBRARY_PATH)
+            p, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+            sigs = {
+                "skinny_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+                "skinny_version": (ctypes.c_int, []),
+                "skinny_nvfp4_packed_bytes": (sz, [i64, i64, ctypes.POINTER(sz)]),
+                "skinny_pack_nvfp4": (ctypes.c_int, [p, p, i64, i64, p, p]),
+                "skinny_unpack_nvfp4": (ctypes.c_int, [p, p, i64, i64, p, p]),
+                "skinny_fp8_packed_bytes": (sz, [i64, i64]),
+                "skinny_pack_fp8": (ctypes.c_int, [p, i64, i64, p]),
+                "skinny_unpack_fp8": (ctypes.c_int, [p, i64, i64, p]),
+                "skinny_workspace_bytes": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.POINTER(sz)]),
+                "skinny_nvfp4_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, ctypes.c_float, i64, p, ctypes.c_int,
+                                                     p, sz, p]),
+                "skinny_fp8_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, i64, p, ctypes.c_int, p, sz, p]),
+                "skinny_device_error": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]),
+            }
+            for name, (res, args) in sigs.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().skinny_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise SkinnyError(status, what)
+
+
+def _np_ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+# ---------------------------------------------------------------------------
+# Host-side packing
+# ---------------------------------------------------------------------------
+
+def nvfp4_packed_bytes(N: int, K: int):
+    """(code bytes, scale bytes) of the packed NVFP4 layout."""
+    sb = ctypes.c_size_t(0)
+    cb = library().skinny_nvfp4_packed_bytes(int(N), int(K), ctypes.byref(sb))
+    return int(cb), int(sb.value)
+
+
+def fp8_packed_bytes(N: int, K: int) -> int:
+    return int(library().skinny_fp8_packed_bytes(int(N), int(K)))
+
+
+def pack_nvfp4(codes: np.ndarray, scales: np.ndarray):
+    """Logical codes [N, K/2] (low nibble = even k) and UE4M3 scales [N, K/16] ->
+    (packed codes, packed scales), both uint8 numpy arrays."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    N, K = codes.shape[0], codes.shape[1] * 2
+    if scales.shape != (N, K // 16):
+        raise ValueError("scales must be [N, K/16]")
+    cb, sb = nvfp4_packed_bytes(N, K)
+    if cb == 0:
+        raise SkinnyError(ERR_INVALID_ARG, "pack_nvfp4 shape")
+    out, sout = np.empty(cb, np.uint8), np.empty(sb, np.uint8)
+    _check(library().skinny_pack_nvfp4(_np_ptr(codes), _np_ptr(scales), N, K, _np_ptr(out), _np_ptr(sout)),
+           "skinny_pack_nvfp4")
+    return out, sout
+
+
+def unpack_nvfp4(packed: np.ndarray, pscales: np.ndarray, N: int, K: int):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    pscales = np.ascontiguousarray(pscales, dtype=np.uint8)
+    codes, scales = np.empty((N, K // 2), np.uint8), np.empty((N, K // 16), np.uint8)
+    _check(library().skinny_unpack_nvfp4(_np_ptr(packed), _np_ptr(pscales), N, K, _np_ptr(codes), _np_ptr(scales)),
+           "skinny_unpack_nvfp4")
+    return codes, scales
+
+
+def pack_fp8(q: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    N, K = q.shape
+    nb = fp8_packed_bytes(N, K)
+    if nb == 0:
+        raise SkinnyError(ERR_INVALID_ARG, "pack_fp8 shape")
+    out = np.empty(nb, np.uint8)
+    _check(library().skinny_pack_fp8(_np_ptr(q), N, K, _np_ptr(out)), "skinny_pack_fp8")
+    return out
+
+
+def unpack_fp8(packed: np.ndarray, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    q = np.empty((N, K), np.uint8)
+    _check(library().skinny_unpack_fp8(_np_ptr(packed), N, K, _np_ptr(q)), "skinny_unpack_fp8")
+    return q
+
+
+# ---------------------------------------------------------------------------
+# Device GEMMs (torch supplies device memory and the stream)
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PackedNVFP4:
+    codes: "object"          # torch.uint8 device tensor (packed layout)
+    scales: "object"         # torch.uint8 device tensor (packed layout)
+    global_scale: float
+    N: int
+    K: int
+
+    @classmethod
+    def from_logical(cls, codes: np.ndarray, scales: np.ndarray, global_scale: float, device="cuda"):
+        import torch
+
+        pc, ps = pack_nvfp4(codes, scales)
+        return cls(torch.from_numpy(pc).to(device), torch.from_numpy(ps).to(device), float(global_scale),
+                   codes.shape[0], codes.shape[1] * 2)
+
+    @property
+    def fmt(self) -> int:
+        return FMT_NVFP4
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.codes.numel() + self.scales.numel())
+
+
+@dataclasses.dataclass
+class PackedFP8:
+    codes: "object"          # torch.uint8 device tensor (packed layout)
+    channel_scale: "object"  # torch.float32 device tensor [N]
+    N: int
+    K: int
+
+    @classmethod
+    def from_logical(cls, q: np.ndarray, channel_scale: np.ndarray, device="cuda"):
+        import torch
+
+        return cls(torch.from_numpy(pack_fp8(q)).to(device),
+                   torch.from_numpy(np.ascontiguousarray(channel_scale, np.float32)).to(device), q.shape[0], q.shape[1])
+
+    @property
+    def fmt(self) -> int:
+        return FMT_FP8
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.codes.numel() + 4 * self.channel_scale.numel())
+
+
+def workspace_bytes(fmt: int, M: int, N: int, K: int) -> int:
+    """Split-K workspace size for one GEMM on the current device."""
+    b = ctypes.c_size_t(0)
+    _check(library().skinny_workspace_bytes(int(fmt), int(M), int(N), int(K), ctypes.byref(b)),
+           "skinny_workspace_bytes")
+    return int(b.value)
+
+
+def make_workspace(fmt: int, M: int, N: int, K: int, device="cuda"):
+    """A zero-filled workspace (its arrival counters must start at zero)."""
+    import torch
+
+    return torch.zeros(workspace_bytes(fmt, M, N, K), dtype=torch.uint8, device=device)
+
+
+def _stream_handle(stream) -> int:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def gemm_into(y, x, w, workspace=None, stream=None) -> None:
+    """y[M, N] = x[M, K] . W^T on the device (y float16 or float32, preallocated)."""
+    import torch
+
+    M, K = x.shape
+    if x.dtype != torch.float16 or not x.is_contiguous() or K != w.K:
+        raise ValueError("x must be a contiguous float16 [M, %d] tensor" % w.K)
+    if y.shape != (M, w.N) or not y.is_contiguous() or y.dtype not in (torch.float16, torch.float32):
+        raise ValueError("y must be a contiguous float16/float32 [M, N] tensor")
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_F16
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    h = _stream_handle(stream)
+    lib = library()
+    if w.fmt == FMT_NVFP4:
+        st = lib.skinny_nvfp4_gemm(x.data_ptr(), M, K, w.codes.data_ptr(), w.scales.data_ptr(),
+                                   ctypes.c_float(w.global_scale), w.N, y.data_ptr(), out, ws_ptr, ws_bytes, h)
+        _check(st, "skinny_nvfp4_gemm")
+    else:
+        st = lib.skinny_fp8_gemm(x.data_ptr(), M, K, w.codes.data_ptr(), w.channel_scale.data_ptr(), w.N,
+                                 y.data_ptr(), out, ws_ptr, ws_bytes, h)
+        _check(st, "skinny_fp8_gemm")
+
+
+def gemm(x, w, out_dtype=None, workspace=None, stream=None):
+    """Allocate y and compute y = x . W^T (float16 output unless out_dtype says otherwise)."""
+    import torch
+
+    y = torch.empty((x.shape[0], w.N), dtype=out_dtype or torch.float16, device=x.device)
+    gemm_into(y, x, w, workspace=workspace, stream=stream)
+    return y
+
+
+def device_error(clear: bool = True) -> int:
+    """Synchronise and read the device-side error word (0 = no wait gave up)."""
+    v = ctypes.c_uint(0)
+    _check(library().skinny_device_error(1 if clear else 0, ctypes.byref(v)), "skinny_device_error")
+    return int(v.value)

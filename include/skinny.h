@@ -1,0 +1,177 @@
+/*
+ * skinny.h -- C ABI of the B200 weight-only skinny GEMM library (libskinny.so).
+ *
+ *   y[M,N] = x[M,K] . W^T,   M = 1..8 rows, W kept compressed in HBM.
+ *
+ * The operation.  During single-request decode (one token, or a k=7
+ * speculative-verify round plus its base token: 8 rows), a language model's
+ * linear layers read far more weight bytes than anything else.  The
+ * v100-skinny pages describe kernels that keep those weights compressed when
+ * they are read from HBM and turn them into FP16 in registers, in small
+ * pieces, against FP16 activations -- "QPN2" for NVFP4 regions of the
+ * checkpoint and "QPN8" for FP8 regions, with the 8-row verify round as the
+ * M=8 case (taozi.news article on v100-skinny, sections "自研 QPN 内核" and
+ * "v1.1 的关键改进"; aiwitness.kr post, section "내가 실제로 만든 것").  This
+ * library is a from-scratch sm_100a implementation of that operation:
+ *
+ *   NVFP4:  W[n][k] = e2m1(code[n][k]) * ue4m3(scale[n][k/16]) * global_scale
+ *   FP8:    W[n][k] = e4m3(q[n][k]) * channel_scale[n]
+ *   y[m][n] = sum_k W[n][k] * x[m][k]     (x FP16, FP32 accumulation)
+ *
+ * E2M1 / E4M3 are the OCP microscaling / OFP8 encodings; NVFP4 groups 16
+ * consecutive K elements under one unsigned E4M3 (UE4M3) scale and adds one
+ * FP32 per-tensor scale.  The dequantised weight matrix never exists in
+ * memory: no N x K FP16 copy is ever made.
+ *
+ * Conventions for every function below:
+ *   - Return value: SKINNY_OK (0) or a negative skinny_status.  Nothing
+ *     aborts or prints; skinny_status_string() names a status.
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     device memory and keeps no per-call state; it caches the SM count and
+ *     kernel attributes per device.
+ *   - "host" pointers are ordinary CPU memory; "device" pointers are global
+ *     memory of the current CUDA device.
+ *   - Layouts are row-major and contiguous: x is [M][K] (leading dim K),
+ *     y is [M][N] (leading dim N), W is [N][K] (the nn.Linear convention).
+ *   - GEMM calls are asynchronous on `stream` (a cudaStream_t, 0 = legacy
+ *     default stream).  Their status covers the argument checks and the
+ *     launch only; a fault inside a kernel appears on the stream as usual and
+ *     a device-side wait that gave up is reported by skinny_device_error().
+ */
+#ifndef SKINNY_H
+#define SKINNY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SKINNY_OK = 0,
+    SKINNY_ERR_INVALID_ARG = -1,  /* null pointer, K % 16 != 0, N or K <= 0, bad dtype, bad scale byte */
+    SKINNY_ERR_UNSUPPORTED = -2,  /* M outside [1, 8], or a size past the library's limits */
+    SKINNY_ERR_ALIGNMENT = -3,    /* a device pointer is not aligned as documented */
+    SKINNY_ERR_CUDA = -4,         /* a CUDA runtime call failed (launch, attribute, device query) */
+    SKINNY_ERR_WORKSPACE = -5     /* workspace non-null but smaller than skinny_workspace_bytes() */
+} skinny_status;
+
+typedef enum { SKINNY_OUT_F16 = 0, SKINNY_OUT_F32 = 1 } skinny_out_dtype;
+
+typedef enum { SKINNY_FMT_NVFP4 = 0, SKINNY_FMT_FP8 = 1 } skinny_format;
+
+#define SKINNY_MAX_M 8
+
+/* Name of a skinny_status value ("SKINNY_OK", ...); never NULL. */
+const char* skinny_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int skinny_version(void);
+
+/* ------------------------------------------------------------------------
+ * Host-side layout routines (pure CPU, no CUDA call).
+ *
+ * The kernels read W in a private tiled order so that each 16 KB tile of
+ * 256 output rows is one contiguous bulk copy and each lane of a warp finds
+ * its tensor-core operand bytes in one 16-byte word.  Rows are padded to a
+ * multiple of 256 and K to a multiple of 128 (NVFP4) or 64 (FP8) with zero
+ * codes and zero scales, which contribute nothing.  The caller packs once per
+ * weight and copies the result to the device.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of the packed NVFP4 code buffer for an N x K weight; the packed scale
+ * buffer's size goes to *scale_bytes (may be NULL).  Returns 0 if N <= 0,
+ * K <= 0 or K % 16 != 0. */
+size_t skinny_nvfp4_packed_bytes(int64_t N, int64_t K, size_t* scale_bytes);
+
+/* Pack a logical NVFP4 tensor.
+ *   codes      host [N][K/2] bytes; element k of row n is in byte k/2, the low
+ *              nibble holding even k and the high nibble odd k (E2M1 codes).
+ *   scales     host [N][K/16] UE4M3 bytes, one per 16 consecutive k.
+ *   w_packed   host, skinny_nvfp4_packed_bytes() bytes, written fully.
+ *   w_scales   host, *scale_bytes bytes, written fully.
+ * Errors: SKINNY_ERR_INVALID_ARG for null pointers, bad sizes, or a scale
+ * byte that is not a finite non-negative UE4M3 value (sign bit set, or the
+ * NaN pattern 0x7F).  Nothing is written on error. */
+int skinny_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, int64_t N, int64_t K,
+                      void* w_packed, void* w_scales);
+
+/* Inverse of skinny_pack_nvfp4 (host only; for tests and tooling). */
+int skinny_unpack_nvfp4(const void* w_packed, const void* w_scales, int64_t N, int64_t K,
+                        uint8_t* codes, uint8_t* scales);
+
+/* Bytes of the packed FP8 buffer for an N x K weight; 0 if N <= 0, K <= 0 or
+ * K % 16 != 0. */
+size_t skinny_fp8_packed_bytes(int64_t N, int64_t K);
+
+/* Pack a logical FP8 tensor: q host [N][K] E4M3 bytes -> w_packed host.
+ * SKINNY_ERR_INVALID_ARG for null pointers, bad sizes, or a NaN code
+ * (0x7F / 0xFF).  The per-channel scales are not packed: they are passed to
+ * skinny_fp8_gemm as a plain float[N] device array. */
+int skinny_pack_fp8(const uint8_t* q, int64_t N, int64_t K, void* w_packed);
+
+/* Inverse of skinny_pack_fp8 (host only). */
+int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
+
+/* ------------------------------------------------------------------------
+ * Device GEMMs.
+ * ---------------------------------------------------------------------- */
+
+/* Size of the optional split-K workspace for one GEMM of this format and
+ * shape on the CURRENT device (it depends on the SM count).  A workspace lets
+ * the kernel split K across CTAs so that every SM streams the same number of
+ * weight bytes (a short-N shape such as 5120 x 5120 has too few 256-row tiles
+ * to fill 148 SMs otherwise).  It holds FP32 partial sums followed by one
+ * arrival counter per 256-row tile; the counters must be ZERO before the
+ * first use and every completed call leaves them zero again, so zero-fill the
+ * workspace once (cudaMemset) and reuse it.  Its layout is the same for every
+ * shape on a device, so a workspace sized for the largest call serves calls of
+ * any shape in turn; it must not be shared by calls that can run at the same
+ * time.
+ * Returns SKINNY_OK and *bytes, or SKINNY_ERR_INVALID_ARG / _CUDA. */
+int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
+
+/* NVFP4 weight-only GEMM: y = x . W^T with W from skinny_pack_nvfp4.
+ *   x            device [M][K] FP16, 16-byte aligned.
+ *   M            1..8 (rows of x: tokens of one decode / verify round).
+ *   K            multiple of 16.
+ *   w_packed     device, packed codes, 16-byte aligned.
+ *   w_scales     device, packed UE4M3 scales, 16-byte aligned.
+ *   global_scale FP32 per-tensor scale, applied to the FP32 sum.
+ *   N            output features.
+ *   y            device [M][N], FP16 (RNE) or FP32 per out_dtype, 4-byte aligned.
+ *   workspace    device or NULL; if non-NULL, at least
+ *                skinny_workspace_bytes(SKINNY_FMT_NVFP4, M, N, K) bytes,
+ *                16-byte aligned, counters zero (see above).  NULL selects
+ *                whole-tile scheduling (no split-K, nothing written besides y).
+ *   stream       cudaStream_t.
+ * Rounding: products of decoded weights and x are exact; only the FP32
+ * summation order differs from exact arithmetic, and it is fixed, so results
+ * are bitwise reproducible run to run for a given shape and device.
+ * Errors: see skinny_status. */
+int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_packed, const void* w_scales,
+                      float global_scale, int64_t N, void* y, int out_dtype, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* FP8 (E4M3) weight-only GEMM with a per-output-channel FP32 scale.
+ *   w_packed       device, from skinny_pack_fp8, 16-byte aligned.
+ *   channel_scale  device float[N], 4-byte aligned.
+ * Other arguments as skinny_nvfp4_gemm (workspace sized with SKINNY_FMT_FP8). */
+int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
+                    const float* channel_scale, int64_t N, void* y, int out_dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device-side error word of the current device.  Every wait inside the
+ * kernels is bounded; a wait that gives up sets a bit here instead of
+ * hanging (1 = consumer wait, 2 = producer wait, 4 = drain wait) and its CTA
+ * returns early, leaving y incomplete.  Synchronises the device, stores the
+ * word in *flags and, if clear != 0, resets it.  Returns SKINNY_OK or
+ * SKINNY_ERR_CUDA. */
+int skinny_device_error(int clear, unsigned* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKINNY_H */

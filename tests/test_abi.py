@@ -1,0 +1,82 @@
+"""The C-ABI library loads and exports every function include/skinny.h declares;
+argument checks that run before any CUDA call return the documented status."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_weight_only_w4a16_b200 as sk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(skinny_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(sk.LIBRARY_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    assert sk.status_string(0) == "SKINNY_OK"
+    assert sk.status_string(-3) == "SKINNY_ERR_ALIGNMENT"
+    assert sk.status_string(-99) == "SKINNY_ERR_UNKNOWN"
+    assert sk.library().skinny_version() >= 100
+
+
+ALIGNED = 1 << 20  # a fake, 16-byte aligned address: never dereferenced by these checks
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), sk.ERR_INVALID_ARG),
+    (dict(y=None), sk.ERR_INVALID_ARG),
+    (dict(w=None), sk.ERR_INVALID_ARG),
+    (dict(M=0), sk.ERR_UNSUPPORTED),
+    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(K=24), sk.ERR_INVALID_ARG),
+    (dict(K=0), sk.ERR_INVALID_ARG),
+    (dict(N=0), sk.ERR_INVALID_ARG),
+    (dict(out=7), sk.ERR_INVALID_ARG),
+    (dict(x=ALIGNED + 8), sk.ERR_ALIGNMENT),
+    (dict(w=ALIGNED + 4), sk.ERR_ALIGNMENT),
+    (dict(ws=ALIGNED + 8), sk.ERR_ALIGNMENT),
+])
+def test_nvfp4_argument_checks(kw, status):
+    a = dict(x=ALIGNED, M=1, K=64, w=ALIGNED, s=ALIGNED, N=32, y=ALIGNED, out=0, ws=None)
+    a.update(kw)
+    st = sk.library().skinny_nvfp4_gemm(a["x"], a["M"], a["K"], a["w"], a["s"], 1.0, a["N"], a["y"], a["out"],
+                                        a["ws"], 0, None)
+    assert st == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(scale=None), sk.ERR_INVALID_ARG),
+    (dict(scale=ALIGNED + 2), sk.ERR_ALIGNMENT),
+    (dict(M=12), sk.ERR_UNSUPPORTED),
+])
+def test_fp8_argument_checks(kw, status):
+    a = dict(x=ALIGNED, M=2, K=64, w=ALIGNED, scale=ALIGNED, N=32, y=ALIGNED)
+    a.update(kw)
+    st = sk.library().skinny_fp8_gemm(a["x"], a["M"], a["K"], a["w"], a["scale"], a["N"], a["y"], 0, None, 0, None)
+    assert st == status
+
+
+def test_workspace_query_argument_checks():
+    b = ctypes.c_size_t(0)
+    lib = sk.library()
+    assert lib.skinny_workspace_bytes(5, 1, 64, 64, ctypes.byref(b)) == sk.ERR_INVALID_ARG
+    assert lib.skinny_workspace_bytes(0, 1, 64, 40, ctypes.byref(b)) == sk.ERR_INVALID_ARG
+    assert lib.skinny_workspace_bytes(0, 9, 64, 64, ctypes.byref(b)) == sk.ERR_UNSUPPORTED
+    assert lib.skinny_workspace_bytes(0, 1, 64, 64, None) == sk.ERR_INVALID_ARG
