@@ -318,10 +318,15 @@ def _oracle_bytes(items) -> int:
 
 
 def oracle_sample_frac(target_s: float, threads: int) -> float:
-    probe = 1.0 / 2048
-    t = _oracle_run(_oracle_inputs(probe), threads)
-    frac = probe * target_s / max(t, 1e-3)
-    return float(min(1.0, max(probe, frac)))
+    """Row fraction whose oracle time is about target_s (two probes, so that the
+    fixed per-call cost of the first does not skew the estimate)."""
+    frac = 1.0 / 1024
+    for _ in range(2):
+        t = _oracle_run(_oracle_inputs(frac), threads)
+        frac = float(min(1.0, max(1.0 / 4096, frac * target_s / max(t, 1e-3))))
+        if t > 0.25 * target_s:
+            break
+    return frac
 
 
 def cpu_baseline(target_s: float = 12.0):
@@ -364,6 +369,39 @@ def reference_arm(args):
     return 0
 
 
+def single_gemm(args):
+    """Time one GEMM of the workload alone (direct launches, rotating weight
+    copies): the small case that ncu captures are taken on."""
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    name, M = args.single.split(":")
+    M = int(M)
+    idx = [s.name for s in si.MIXED_LAYER].index(name)
+    spec = si.MIXED_LAYER[idx]
+    torch.cuda.set_device(0)
+    weights, xs, ys, ws = build_device_workload(torch.device("cuda", 0))
+    if M not in xs:
+        xs[M] = [torch.from_numpy(si.activations(M, s.K, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=100 + i)).cuda()
+                 for i, s in enumerate(si.MIXED_LAYER)]
+        ys[M] = [torch.empty((M, s.N), dtype=torch.float16, device="cuda") for s in si.MIXED_LAYER]
+    for i in range(args.warmup):
+        sk.gemm_into(ys[M][idx], xs[M][idx], weights[i % COPIES][idx], workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        sk.gemm_into(ys[M][idx], xs[M][idx], weights[i % COPIES][idx], workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / args.steps
+    b = gemm_bytes(spec, M)
+    print(json.dumps({"single": args.single, "us_per_launch": round(us, 3), "GB/s": round(b / us / 1e3, 1),
+                      "alg_bytes": b}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------------------
 # Main (our arm)
 # ---------------------------------------------------------------------------
@@ -376,12 +414,15 @@ def main(argv=None):
     ap.add_argument("--impl", default="skinny", choices=["skinny", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--event-rounds", type=int, default=20)
+    ap.add_argument("--single", default=None, help="NAME:M -- time one GEMM of the workload alone")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     if args.impl == "reference":
         return reference_arm(args)
+    if args.single:
+        return single_gemm(args)
 
     import torch
     import torch.distributed as dist
