@@ -66,6 +66,9 @@ def library() -> ctypes.CDLL:
                                                      p, sz, p]),
                 "skinny_fp8_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, i64, p, ctypes.c_int, p, sz, p]),
                 "skinny_device_error": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]),
+                "skinny_nvfp4_gemm_static_ws": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, ctypes.c_float, i64, p,
+                                                               ctypes.c_int, p]),
+                "skinny_static_workspace_capacity": (sz, []),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(lib, name)

@@ -499,6 +499,69 @@ extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_pa
     return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 GEMM with split-K scratch in a static device array, for callers that
+// cannot allocate device memory.
+// ---------------------------------------------------------------------------
+
+namespace skinny {
+
+// 4 MiB of split-K scratch per device, reserved when the library's device code
+// is loaded on that device and held until the process exits.
+constexpr size_t kStaticWorkspaceBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_static_workspace on each device.  In host code the
+// array's name only stands in for the symbol, so the address is looked up with
+// cudaGetSymbolAddress, once per device, while that device is current.
+static void* g_static_workspace_addr[kMaxDevices];
+
+static int static_workspace_address(void** addr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SKINNY_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_static_workspace_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return SKINNY_ERR_CUDA;
+        g_static_workspace_addr[dev] = p;
+    }
+    *addr = g_static_workspace_addr[dev];
+    return SKINNY_OK;
+}
+
+}  // namespace skinny
+
+extern "C" size_t skinny_static_workspace_capacity(void) { return kStaticWorkspaceBytes; }
+
+extern "C" int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, const void* w_packed,
+                                           const void* w_scales, float global_scale, int64_t N, void* y,
+                                           int out_dtype, void* stream)
+{
+    int rc = check_common(x, M, K, N, y, out_dtype, nullptr);
+    if (rc != SKINNY_OK) return rc;
+    if (!w_packed || !w_scales) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(w_packed, 16) || !aligned(w_scales, 16)) return SKINNY_ERR_ALIGNMENT;
+    int sms = 0;
+    rc = current_device(&sms);
+    if (rc != SKINNY_OK) return rc;
+    Plan pl;
+    rc = make_plan(SKINNY_FMT_NVFP4, N, K, sms, true, &pl);
+    if (rc != SKINNY_OK) return rc;
+    if (pl.workspace_bytes > kStaticWorkspaceBytes) return SKINNY_ERR_UNSUPPORTED;
+    void* ws = nullptr;
+    rc = static_workspace_address(&ws);
+    if (rc != SKINNY_OK) return rc;
+    // The array keeps whatever the previous call left; the arrival counters of
+    // this call must start at zero, so clear them on the call's stream.
+    const size_t counter_bytes = pl.workspace_bytes - pl.partial_bytes;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + pl.partial_bytes, 0, counter_bytes, st) != cudaSuccess)
+        return SKINNY_ERR_CUDA;
+    return skinny_nvfp4_gemm(x, M, K, w_packed, w_scales, global_scale, N, y, out_dtype, ws, kStaticWorkspaceBytes,
+                             stream);
+}
+
 extern "C" int skinny_device_error(int clear, unsigned* flags)
 {
     if (!flags) return SKINNY_ERR_INVALID_ARG;

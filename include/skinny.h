@@ -162,6 +162,36 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
                     const float* channel_scale, int64_t N, void* y, int out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* NVFP4 GEMM for callers that cannot allocate device memory.
+ *
+ * There is no counterpart of this entry point on the v100-skinny pages; it
+ * exists for code that may not call cudaMalloc -- for example a serving
+ * engine that has handed all free HBM to its own pool (KV cache and weights)
+ * and forbids raw allocations, a plugin running inside a host framework that
+ * gives it no allocator, or a latency-critical caller that must not hit
+ * cudaMalloc's implicit device synchronisation.
+ *
+ * It computes exactly what skinny_nvfp4_gemm computes with a workspace (same
+ * kernel, same split-K schedule, same arguments and errors), but its split-K
+ * scratch lives in one static device array of skinny_static_workspace_capacity()
+ * bytes (4 MiB) that every GPU which loads this library holds until the
+ * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.  Shapes whose scratch would not fit (more than
+ * about 442k 256-row tiles on a 148-SM B200) return SKINNY_ERR_UNSUPPORTED.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, which may load the library's device code); make that
+ * first call outside any stream capture.  Every call enqueues, on `stream`, a
+ * clear of the arrival counters it uses, then the GEMM.  All calls on a device
+ * share the one array, so calls that can overlap on the GPU (different
+ * streams, or concurrent graph branches) race and corrupt each other's
+ * results: serialise them. */
+int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, const void* w_packed, const void* w_scales,
+                                float global_scale, int64_t N, void* y, int out_dtype, void* stream);
+
+/* Size in bytes of the static scratch array used by skinny_nvfp4_gemm_static_ws. */
+size_t skinny_static_workspace_capacity(void);
+
 /* Device-side error word of the current device.  Every wait inside the
  * kernels is bounded; a wait that gives up sets a bit here instead of
  * hanging (1 = consumer wait, 2 = producer wait, 4 = drain wait) and its CTA
