@@ -159,11 +159,9 @@ def build_device_workload(dev):
     for i, spec in enumerate(si.MIXED_LAYER):
         logical = si.weights_for(spec, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=10 * i)
         if spec.fmt == "nvfp4":
-            pc, ps = sk.pack_nvfp4(*logical)
-            base = (torch.from_numpy(pc).to(dev), torch.from_numpy(ps).to(dev))
+            base = torch.from_numpy(sk.pack_nvfp4(*logical)).to(dev)
             for c in range(COPIES):
-                cc, cs = (base[0], base[1]) if c == 0 else (base[0].clone(), base[1].clone())
-                weights[c].append(sk.PackedNVFP4(cc, cs, spec.global_scale, spec.N, spec.K))
+                weights[c].append(sk.PackedNVFP4(base if c == 0 else base.clone(), spec.global_scale, spec.N, spec.K))
         else:
             pc = torch.from_numpy(sk.pack_fp8(logical[0])).to(dev)
             s = torch.from_numpy(logical[1]).to(dev)

@@ -55,18 +55,18 @@ def library() -> ctypes.CDLL:
             sigs = {
                 "skinny_status_string": (ctypes.c_char_p, [ctypes.c_int]),
                 "skinny_version": (ctypes.c_int, []),
-                "skinny_nvfp4_packed_bytes": (sz, [i64, i64, ctypes.POINTER(sz)]),
-                "skinny_pack_nvfp4": (ctypes.c_int, [p, p, i64, i64, p, p]),
-                "skinny_unpack_nvfp4": (ctypes.c_int, [p, p, i64, i64, p, p]),
+                "skinny_nvfp4_packed_bytes": (sz, [i64, i64]),
+                "skinny_pack_nvfp4": (ctypes.c_int, [p, p, i64, i64, p]),
+                "skinny_unpack_nvfp4": (ctypes.c_int, [p, i64, i64, p, p]),
                 "skinny_fp8_packed_bytes": (sz, [i64, i64]),
                 "skinny_pack_fp8": (ctypes.c_int, [p, i64, i64, p]),
                 "skinny_unpack_fp8": (ctypes.c_int, [p, i64, i64, p]),
                 "skinny_workspace_bytes": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, i64, i64, ctypes.POINTER(sz)]),
-                "skinny_nvfp4_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, ctypes.c_float, i64, p, ctypes.c_int,
+                "skinny_nvfp4_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, ctypes.c_int,
                                                      p, sz, p]),
                 "skinny_fp8_gemm": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, i64, p, ctypes.c_int, p, sz, p]),
                 "skinny_device_error": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]),
-                "skinny_nvfp4_gemm_static_ws": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, ctypes.c_float, i64, p,
+                "skinny_nvfp4_gemm_static_ws": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
                                                                ctypes.c_int, p]),
                 "skinny_static_workspace_capacity": (sz, []),
             }
@@ -95,39 +95,35 @@ def _np_ptr(a: np.ndarray) -> int:
 # Host-side packing
 # ---------------------------------------------------------------------------
 
-def nvfp4_packed_bytes(N: int, K: int):
-    """(code bytes, scale bytes) of the packed NVFP4 layout."""
-    sb = ctypes.c_size_t(0)
-    cb = library().skinny_nvfp4_packed_bytes(int(N), int(K), ctypes.byref(sb))
-    return int(cb), int(sb.value)
+def nvfp4_packed_bytes(N: int, K: int) -> int:
+    """Bytes of the packed NVFP4 layout (codes and block scales)."""
+    return int(library().skinny_nvfp4_packed_bytes(int(N), int(K)))
 
 
 def fp8_packed_bytes(N: int, K: int) -> int:
     return int(library().skinny_fp8_packed_bytes(int(N), int(K)))
 
 
-def pack_nvfp4(codes: np.ndarray, scales: np.ndarray):
+def pack_nvfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """Logical codes [N, K/2] (low nibble = even k) and UE4M3 scales [N, K/16] ->
-    (packed codes, packed scales), both uint8 numpy arrays."""
+    the packed uint8 buffer (tiles of codes with their block scales)."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     N, K = codes.shape[0], codes.shape[1] * 2
     if scales.shape != (N, K // 16):
         raise ValueError("scales must be [N, K/16]")
-    cb, sb = nvfp4_packed_bytes(N, K)
-    if cb == 0:
+    nb = nvfp4_packed_bytes(N, K)
+    if nb == 0:
         raise SkinnyError(ERR_INVALID_ARG, "pack_nvfp4 shape")
-    out, sout = np.empty(cb, np.uint8), np.empty(sb, np.uint8)
-    _check(library().skinny_pack_nvfp4(_np_ptr(codes), _np_ptr(scales), N, K, _np_ptr(out), _np_ptr(sout)),
-           "skinny_pack_nvfp4")
-    return out, sout
+    out = np.empty(nb, np.uint8)
+    _check(library().skinny_pack_nvfp4(_np_ptr(codes), _np_ptr(scales), N, K, _np_ptr(out)), "skinny_pack_nvfp4")
+    return out
 
 
-def unpack_nvfp4(packed: np.ndarray, pscales: np.ndarray, N: int, K: int):
+def unpack_nvfp4(packed: np.ndarray, N: int, K: int):
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
-    pscales = np.ascontiguousarray(pscales, dtype=np.uint8)
     codes, scales = np.empty((N, K // 2), np.uint8), np.empty((N, K // 16), np.uint8)
-    _check(library().skinny_unpack_nvfp4(_np_ptr(packed), _np_ptr(pscales), N, K, _np_ptr(codes), _np_ptr(scales)),
+    _check(library().skinny_unpack_nvfp4(_np_ptr(packed), N, K, _np_ptr(codes), _np_ptr(scales)),
            "skinny_unpack_nvfp4")
     return codes, scales
 
@@ -156,8 +152,7 @@ def unpack_fp8(packed: np.ndarray, N: int, K: int) -> np.ndarray:
 
 @dataclasses.dataclass
 class PackedNVFP4:
-    codes: "object"          # torch.uint8 device tensor (packed layout)
-    scales: "object"         # torch.uint8 device tensor (packed layout)
+    data: "object"           # torch.uint8 device tensor (packed tiles: codes + block scales)
     global_scale: float
     N: int
     K: int
@@ -166,9 +161,8 @@ class PackedNVFP4:
     def from_logical(cls, codes: np.ndarray, scales: np.ndarray, global_scale: float, device="cuda"):
         import torch
 
-        pc, ps = pack_nvfp4(codes, scales)
-        return cls(torch.from_numpy(pc).to(device), torch.from_numpy(ps).to(device), float(global_scale),
-                   codes.shape[0], codes.shape[1] * 2)
+        return cls(torch.from_numpy(pack_nvfp4(codes, scales)).to(device), float(global_scale), codes.shape[0],
+                   codes.shape[1] * 2)
 
     @property
     def fmt(self) -> int:
@@ -176,7 +170,7 @@ class PackedNVFP4:
 
     @property
     def nbytes(self) -> int:
-        return int(self.codes.numel() + self.scales.numel())
+        return int(self.data.numel())
 
 
 @dataclasses.dataclass
@@ -240,8 +234,8 @@ def gemm_into(y, x, w, workspace=None, stream=None) -> None:
     h = _stream_handle(stream)
     lib = library()
     if w.fmt == FMT_NVFP4:
-        st = lib.skinny_nvfp4_gemm(x.data_ptr(), M, K, w.codes.data_ptr(), w.scales.data_ptr(),
-                                   ctypes.c_float(w.global_scale), w.N, y.data_ptr(), out, ws_ptr, ws_bytes, h)
+        st = lib.skinny_nvfp4_gemm(x.data_ptr(), M, K, w.data.data_ptr(), ctypes.c_float(w.global_scale), w.N,
+                                   y.data_ptr(), out, ws_ptr, ws_bytes, h)
         _check(st, "skinny_nvfp4_gemm")
     else:
         st = lib.skinny_fp8_gemm(x.data_ptr(), M, K, w.codes.data_ptr(), w.channel_scale.data_ptr(), w.N,

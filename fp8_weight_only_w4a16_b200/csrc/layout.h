@@ -1,22 +1,27 @@
 // layout.h -- the packed weight layout shared by the host packer and the
 // sm_100a kernels (private to libskinny; the public ABI only sees byte counts).
 //
-// A weight matrix W[N][K] is cut into tiles of 256 output rows x TILE_K
-// columns (TILE_K = 128 for NVFP4, 64 for FP8).  Tiles are stored in the
-// order  tile(g, c) = g * C + c  (g = row tile, c = K tile), so one CTA that
-// walks a contiguous range of tiles streams one contiguous byte range.  Every
-// tile is exactly 16384 code bytes (plus 2048 scale bytes for NVFP4, in a
-// separate buffer with the same tile order), i.e. one bulk copy each.
+// Tiles.  W[N][K] is cut into tiles of 256 output rows x 128 columns, stored in
+// the order tile(g, c) = g * C + c (g = row tile, c = K tile), so a CTA that
+// walks a contiguous range of tiles streams one contiguous byte range, and
+// consecutive tiles can be fetched together by one bulk copy.  An NVFP4 tile
+// is 16384 code bytes followed by its 2048 UE4M3 scale bytes (18432 bytes);
+// an FP8 tile is 32768 bytes.
 //
-// Inside a tile, 16 "strips" of 16 rows follow each other; a strip's 64-K
-// chunk is laid out for one warp-wide m16n8k16 tensor-core sequence: lane
-// l = 4*gid + t owns rows {gid, gid+8} of the strip and the 16 logical K
-// values [16t, 16t+16) of the chunk, spread over four k16 MMA steps j = 0..3.
-// MMA k-slot {2t, 2t+1, 2t+8, 2t+9} of step j carries logical k
+// Inside a tile: 16 strips of 16 rows; each strip has two 64-column chunks.
+// One chunk of one strip is laid out for a warp-wide sequence of four
+// m16n8k16 tensor-core steps j = 0..3: lane l = 4*gid + t owns rows
+// {gid, gid+8} of the strip and the 16 logical columns [16t, 16t+16) of the
+// chunk.  MMA k-slot {2t, 2t+1, 2t+8, 2t+9} of step j carries logical column
 // 16t + 4j + {0, 1, 2, 3}; the activations are staged in the same order, so
-// the dot product is unchanged and each lane reads its B operand for all four
-// steps as 32 contiguous bytes.  Register r of the A fragment (r = 0..3)
-// holds row gid + 8*(r&1) at logical k 16t + 4j + 2*(r>>1) + {0, 1}.
+// the dot product is unchanged and a lane reads its B operand for all four
+// steps as 32 contiguous bytes.  Register r of the A fragment (r = 0..3) holds
+// row gid + 8*(r&1) at logical columns 16t + 4j + 2*(r>>1) + {0, 1} (element
+// e = 0 in the low half of the f16x2 register, e = 1 in the high half).
+//
+// NVFP4 words.  A lane's 16 bytes are four 32-bit words, word j feeding MMA
+// step j: byte r holds A register r, element e in nibble e (low nibble first)
+// -- the input of Blackwell's exact cvt.rn.f16x2.e2m1x2.
 #pragma once
 #include <stdint.h>
 
@@ -26,60 +31,71 @@ constexpr int kTileRows = 256;       // output rows per tile
 constexpr int kStripRows = 16;       // rows per MMA strip (the m16 of m16n8k16)
 constexpr int kStrips = kTileRows / kStripRows;
 constexpr int kChunkK = 64;          // K per strip chunk (four k16 steps)
-constexpr int kTileCodeBytes = 16384;
+constexpr int kTileK = 128;          // K per tile: two chunks
+constexpr int kChunks = kTileK / kChunkK;
 
-constexpr int kNvfp4TileK = 128;     // two chunks per NVFP4 tile
-constexpr int kNvfp4TileScaleBytes = kTileRows * kNvfp4TileK / 16;  // 2048
-constexpr int kFp8TileK = 64;        // one chunk per FP8 tile
-
-static_assert(kTileRows * kNvfp4TileK / 2 == kTileCodeBytes, "nvfp4 tile size");
-static_assert(kTileRows * kFp8TileK == kTileCodeBytes, "fp8 tile size");
-
-// cvt.rn.f16x2.e2m1x2 turns the low nibble of its byte into the low half of
-// the f16x2 result, and cvt.rn.f16x2.e4m3x2 turns the low byte of its 16-bit
-// input into the low half.
-constexpr bool kLowFirst = true;
+constexpr int kNvfp4TileCodeBytes = kTileRows * kTileK / 2;       // 16384
+constexpr int kNvfp4TileScaleBytes = kTileRows * kTileK / 16;     // 2048
+constexpr int kNvfp4TileBytes = kNvfp4TileCodeBytes + kNvfp4TileScaleBytes;
+constexpr int kFp8TileBytes = kTileRows * kTileK;                 // 32768
 
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
-// Byte offset, inside a 16384-byte NVFP4 code tile, of the byte that holds the
-// element (row r in 0..255, column k in 0..127); *high = 1 if it is the high
-// nibble.
-inline int nvfp4_code_offset(int r, int k, int* high)
+// Where element (row r in 0..255, column k in 0..127) of a tile lives.
+struct Slot {
+    int word;   // byte offset of its 32-bit word inside the tile's codes
+    int j;      // MMA step (word index inside the lane's 16 / 32 bytes)
+    int reg;    // A-fragment register
+    int e;      // half of the f16x2 register (0 = low)
+};
+
+inline Slot tile_slot(int r, int k)
 {
     const int strip = r / 16, rr = r % 16;
     const int gid = rr % 8, h = rr / 8;
     const int ch = k / 64, kk = k % 64;
     const int t = kk / 16, w = kk % 16;
     const int j = w / 4, o = w % 4;
-    const int reg = h + 2 * (o / 2);
-    const int lane = 4 * gid + t;
-    *high = kLowFirst ? (o % 2) : 1 - (o % 2);
-    return strip * 1024 + ch * 512 + lane * 16 + 4 * j + reg;
+    Slot s;
+    s.j = j;
+    s.reg = h + 2 * (o / 2);
+    s.e = o % 2;
+    s.word = strip * (kChunks * 512) + ch * 512 + (4 * gid + t) * 16 + 4 * j;  // NVFP4 placement
+    return s;
 }
 
-// Byte offset, inside a 2048-byte NVFP4 scale tile, of the UE4M3 scale of row
+// NVFP4: set / read the nibble of slot s in its word.
+inline uint32_t nvfp4_put(uint32_t word, const Slot& s, uint32_t code)
+{
+    return word | (code << (8 * s.reg + 4 * s.e));
+}
+
+inline uint32_t nvfp4_get(uint32_t word, const Slot& s) { return (word >> (8 * s.reg + 4 * s.e)) & 0xFu; }
+
+// Byte offset, inside the 2048 scale bytes of an NVFP4 tile, of the UE4M3 scale of row
 // r (0..255) and 16-column block b (0..7).  A lane reads its two scales (rows
-// gid and gid+8 of its strip, block t of the chunk) as one 16-bit word.
+// gid and gid+8 of its strip, block t of the chunk) as one 16-bit word: row
+// gid in the low byte (cvt.rn.f16x2.e4m3x2 turns the low byte into the low
+// half).
 inline int nvfp4_scale_offset(int r, int b)
 {
     const int strip = r / 16, rr = r % 16;
     const int gid = rr % 8, h = rr / 8;
     const int ch = b / 4, t = b % 4;
-    return strip * 128 + ch * 64 + t * 16 + gid * 2 + (kLowFirst ? h : 1 - h);
+    return strip * 128 + ch * 64 + t * 16 + gid * 2 + h;
 }
 
-// Byte offset, inside a 16384-byte FP8 tile, of element (row r, column k in 0..63).
-inline int fp8_code_offset(int r, int k)
+// Byte offset, inside a 32768-byte FP8 tile, of element (row r, column k).
+// A lane's 32 bytes per chunk: step j in bytes 8j..8j+7, register r in bytes
+// 2r, 2r+1, element e in byte e (cvt.rn.f16x2.e4m3x2 turns the low byte into
+// the low half).
+inline int fp8_offset(int r, int k)
 {
+    const Slot s = tile_slot(r, k);
     const int strip = r / 16, rr = r % 16;
-    const int gid = rr % 8, h = rr / 8;
-    const int t = k / 16, w = k % 16;
-    const int j = w / 4, o = w % 4;
-    const int reg = h + 2 * (o / 2);
-    const int e = kLowFirst ? (o % 2) : 1 - (o % 2);
-    const int lane = 4 * gid + t;
-    return strip * 1024 + lane * 32 + 8 * j + 2 * reg + e;
+    const int gid = rr % 8;
+    const int ch = k / 64, t = (k % 64) / 16;
+    return strip * (kChunks * 1024) + ch * 1024 + (4 * gid + t) * 32 + 8 * s.j + 2 * s.reg + s.e;
 }
 
 }  // namespace skinny

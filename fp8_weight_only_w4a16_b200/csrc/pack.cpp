@@ -2,8 +2,6 @@
 // layout (see layout.h), and the inverse.  Pure CPU code, no CUDA calls.
 #include <string.h>
 
-#include <vector>
-
 #include "../../include/skinny.h"
 #include "layout.h"
 
@@ -13,7 +11,7 @@ namespace {
 
 bool valid_shape(int64_t N, int64_t K)
 {
-    return N > 0 && K > 0 && K % 16 == 0 && N <= (int64_t(1) << 31) && K <= (int64_t(1) << 30);
+    return N > 0 && K > 0 && K % 16 == 0 && N <= (int64_t(1) << 30) && K <= (int64_t(1) << 30);
 }
 
 // A UE4M3 block scale must be finite and non-negative: sign bit clear and not
@@ -22,87 +20,82 @@ bool valid_ue4m3(uint8_t b) { return b < 0x7F; }
 
 bool valid_e4m3(uint8_t b) { return (b & 0x7F) != 0x7F; }
 
+inline uint32_t load_word(const uint8_t* p)
+{
+    uint32_t v;
+    memcpy(&v, p, 4);
+    return v;
+}
+
+inline void store_word(uint8_t* p, uint32_t v) { memcpy(p, &v, 4); }
+
 }  // namespace
 
-extern "C" size_t skinny_nvfp4_packed_bytes(int64_t N, int64_t K, size_t* scale_bytes)
+extern "C" size_t skinny_nvfp4_packed_bytes(int64_t N, int64_t K)
 {
-    if (!valid_shape(N, K)) {
-        if (scale_bytes) *scale_bytes = 0;
-        return 0;
-    }
-    const int64_t Np = round_up(N, kTileRows), Kp = round_up(K, kNvfp4TileK);
-    if (scale_bytes) *scale_bytes = (size_t)(Np * Kp / 16);
-    return (size_t)(Np * Kp / 2);
+    if (!valid_shape(N, K)) return 0;
+    return (size_t)(round_up(N, kTileRows) / kTileRows * (round_up(K, kTileK) / kTileK)) * kNvfp4TileBytes;
 }
 
 extern "C" size_t skinny_fp8_packed_bytes(int64_t N, int64_t K)
 {
     if (!valid_shape(N, K)) return 0;
-    return (size_t)(round_up(N, kTileRows) * round_up(K, kFp8TileK));
+    return (size_t)(round_up(N, kTileRows) * round_up(K, kTileK));
 }
 
 extern "C" int skinny_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, int64_t N, int64_t K,
-                                 void* w_packed, void* w_scales)
+                                 void* w_packed)
 {
-    if (!codes || !scales || !w_packed || !w_scales || !valid_shape(N, K)) return SKINNY_ERR_INVALID_ARG;
+    if (!codes || !scales || !w_packed || !valid_shape(N, K)) return SKINNY_ERR_INVALID_ARG;
     const int64_t nblk = K / 16;
     for (int64_t i = 0; i < N * nblk; ++i)
         if (!valid_ue4m3(scales[i])) return SKINNY_ERR_INVALID_ARG;
 
-    size_t sbytes = 0;
-    const size_t cbytes = skinny_nvfp4_packed_bytes(N, K, &sbytes);
     uint8_t* out = (uint8_t*)w_packed;
-    uint8_t* sout = (uint8_t*)w_scales;
-    memset(out, 0, cbytes);  // padding rows / columns: code 0 (+0.0)
-    memset(sout, 0, sbytes); // padding scales: 0 (the block contributes 0)
+    // padding rows / columns: code 0 (+0.0) and scale 0 (the block contributes 0)
+    memset(out, 0, skinny_nvfp4_packed_bytes(N, K));
 
-    const int64_t C = round_up(K, kNvfp4TileK) / kNvfp4TileK;
+    const int64_t C = round_up(K, kTileK) / kTileK;
     for (int64_t n = 0; n < N; ++n) {
         const int64_t g = n / kTileRows;
         const int r = (int)(n % kTileRows);
         for (int64_t k = 0; k < K; ++k) {
-            const int64_t c = k / kNvfp4TileK;
-            const int kk = (int)(k % kNvfp4TileK);
+            const int64_t c = k / kTileK;
             const uint8_t byte = codes[n * (K / 2) + k / 2];
-            const uint8_t code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
-            int high = 0;
-            const int off = nvfp4_code_offset(r, kk, &high);
-            uint8_t* dst = out + (g * C + c) * kTileCodeBytes + off;
-            *dst |= high ? (uint8_t)(code << 4) : code;
+            const uint32_t code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+            const Slot s = tile_slot(r, (int)(k % kTileK));
+            uint8_t* dst = out + (g * C + c) * kNvfp4TileBytes + s.word;
+            store_word(dst, nvfp4_put(load_word(dst), s, code));
         }
         for (int64_t b = 0; b < nblk; ++b) {
-            const int64_t c = (b * 16) / kNvfp4TileK;
-            const int bb = (int)(b % (kNvfp4TileK / 16));
-            sout[(g * C + c) * kNvfp4TileScaleBytes + nvfp4_scale_offset(r, bb)] = scales[n * nblk + b];
+            const int64_t c = (b * 16) / kTileK;
+            const int bb = (int)(b % (kTileK / 16));
+            out[(g * C + c) * kNvfp4TileBytes + kNvfp4TileCodeBytes + nvfp4_scale_offset(r, bb)] = scales[n * nblk + b];
         }
     }
     return SKINNY_OK;
 }
 
-extern "C" int skinny_unpack_nvfp4(const void* w_packed, const void* w_scales, int64_t N, int64_t K,
-                                   uint8_t* codes, uint8_t* scales)
+extern "C" int skinny_unpack_nvfp4(const void* w_packed, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales)
 {
-    if (!codes || !scales || !w_packed || !w_scales || !valid_shape(N, K)) return SKINNY_ERR_INVALID_ARG;
+    if (!codes || !scales || !w_packed || !valid_shape(N, K)) return SKINNY_ERR_INVALID_ARG;
     const uint8_t* in = (const uint8_t*)w_packed;
-    const uint8_t* sin = (const uint8_t*)w_scales;
-    const int64_t C = round_up(K, kNvfp4TileK) / kNvfp4TileK;
+    const int64_t C = round_up(K, kTileK) / kTileK;
     const int64_t nblk = K / 16;
     memset(codes, 0, (size_t)(N * (K / 2)));
     for (int64_t n = 0; n < N; ++n) {
         const int64_t g = n / kTileRows;
         const int r = (int)(n % kTileRows);
         for (int64_t k = 0; k < K; ++k) {
-            const int64_t c = k / kNvfp4TileK;
-            int high = 0;
-            const int off = nvfp4_code_offset(r, (int)(k % kNvfp4TileK), &high);
-            const uint8_t byte = in[(g * C + c) * kTileCodeBytes + off];
-            const uint8_t code = high ? (byte >> 4) : (byte & 0x0F);
-            codes[n * (K / 2) + k / 2] |= (k % 2 == 0) ? code : (uint8_t)(code << 4);
+            const int64_t c = k / kTileK;
+            const Slot s = tile_slot(r, (int)(k % kTileK));
+            const uint32_t code = nvfp4_get(load_word(in + (g * C + c) * kNvfp4TileBytes + s.word), s);
+            codes[n * (K / 2) + k / 2] |= (k % 2 == 0) ? (uint8_t)code : (uint8_t)(code << 4);
         }
         for (int64_t b = 0; b < nblk; ++b) {
-            const int64_t c = (b * 16) / kNvfp4TileK;
-            scales[n * nblk + b] =
-                sin[(g * C + c) * kNvfp4TileScaleBytes + nvfp4_scale_offset(r, (int)(b % (kNvfp4TileK / 16)))];
+            const int64_t c = (b * 16) / kTileK;
+            scales[n * nblk + b] = in[(g * C + c) * kNvfp4TileBytes + kNvfp4TileCodeBytes +
+                                      nvfp4_scale_offset(r, (int)(b % (kTileK / 16)))];
         }
     }
     return SKINNY_OK;
@@ -115,13 +108,13 @@ extern "C" int skinny_pack_fp8(const uint8_t* q, int64_t N, int64_t K, void* w_p
         if (!valid_e4m3(q[i])) return SKINNY_ERR_INVALID_ARG;
     uint8_t* out = (uint8_t*)w_packed;
     memset(out, 0, skinny_fp8_packed_bytes(N, K));
-    const int64_t C = round_up(K, kFp8TileK) / kFp8TileK;
+    const int64_t C = round_up(K, kTileK) / kTileK;
     for (int64_t n = 0; n < N; ++n) {
         const int64_t g = n / kTileRows;
         const int r = (int)(n % kTileRows);
         for (int64_t k = 0; k < K; ++k) {
-            const int64_t c = k / kFp8TileK;
-            out[(g * C + c) * kTileCodeBytes + fp8_code_offset(r, (int)(k % kFp8TileK))] = q[n * K + k];
+            const int64_t c = k / kTileK;
+            out[(g * C + c) * kFp8TileBytes + fp8_offset(r, (int)(k % kTileK))] = q[n * K + k];
         }
     }
     return SKINNY_OK;
@@ -131,13 +124,13 @@ extern "C" int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uin
 {
     if (!q || !w_packed || !valid_shape(N, K)) return SKINNY_ERR_INVALID_ARG;
     const uint8_t* in = (const uint8_t*)w_packed;
-    const int64_t C = round_up(K, kFp8TileK) / kFp8TileK;
+    const int64_t C = round_up(K, kTileK) / kTileK;
     for (int64_t n = 0; n < N; ++n) {
         const int64_t g = n / kTileRows;
         const int r = (int)(n % kTileRows);
         for (int64_t k = 0; k < K; ++k) {
-            const int64_t c = k / kFp8TileK;
-            q[n * K + k] = in[(g * C + c) * kTileCodeBytes + fp8_code_offset(r, (int)(k % kFp8TileK))];
+            const int64_t c = k / kTileK;
+            q[n * K + k] = in[(g * C + c) * kFp8TileBytes + fp8_offset(r, (int)(k % kTileK))];
         }
     }
     return SKINNY_OK;

@@ -72,34 +72,32 @@ int skinny_version(void);
 /* ------------------------------------------------------------------------
  * Host-side layout routines (pure CPU, no CUDA call).
  *
- * The kernels read W in a private tiled order so that each 16 KB tile of
- * 256 output rows is one contiguous bulk copy and each lane of a warp finds
- * its tensor-core operand bytes in one 16-byte word.  Rows are padded to a
- * multiple of 256 and K to a multiple of 128 (NVFP4) or 64 (FP8) with zero
- * codes and zero scales, which contribute nothing.  The caller packs once per
- * weight and copies the result to the device.
+ * The kernels read W in a private tiled order: tiles of 256 output rows x
+ * 128 columns, consecutive in memory along K then N, so that a run of tiles is
+ * one contiguous bulk copy and each lane of a warp finds its tensor-core
+ * operand bytes in one 16-byte word.  An NVFP4 tile carries its UE4M3 block
+ * scales (16 KB codes + 2 KB scales); an FP8 tile is 32 KB.  Rows are padded
+ * to a multiple of 256 and K to a multiple of 128 with zero codes and zero
+ * scales, which contribute nothing.  The caller packs once per weight and
+ * copies the result to the device.
  * ---------------------------------------------------------------------- */
 
-/* Bytes of the packed NVFP4 code buffer for an N x K weight; the packed scale
- * buffer's size goes to *scale_bytes (may be NULL).  Returns 0 if N <= 0,
- * K <= 0 or K % 16 != 0. */
-size_t skinny_nvfp4_packed_bytes(int64_t N, int64_t K, size_t* scale_bytes);
+/* Bytes of the packed NVFP4 buffer (codes and block scales) for an N x K
+ * weight.  Returns 0 if N <= 0, K <= 0 or K % 16 != 0. */
+size_t skinny_nvfp4_packed_bytes(int64_t N, int64_t K);
 
 /* Pack a logical NVFP4 tensor.
  *   codes      host [N][K/2] bytes; element k of row n is in byte k/2, the low
  *              nibble holding even k and the high nibble odd k (E2M1 codes).
  *   scales     host [N][K/16] UE4M3 bytes, one per 16 consecutive k.
  *   w_packed   host, skinny_nvfp4_packed_bytes() bytes, written fully.
- *   w_scales   host, *scale_bytes bytes, written fully.
  * Errors: SKINNY_ERR_INVALID_ARG for null pointers, bad sizes, or a scale
  * byte that is not a finite non-negative UE4M3 value (sign bit set, or the
  * NaN pattern 0x7F).  Nothing is written on error. */
-int skinny_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, int64_t N, int64_t K,
-                      void* w_packed, void* w_scales);
+int skinny_pack_nvfp4(const uint8_t* codes, const uint8_t* scales, int64_t N, int64_t K, void* w_packed);
 
 /* Inverse of skinny_pack_nvfp4 (host only; for tests and tooling). */
-int skinny_unpack_nvfp4(const void* w_packed, const void* w_scales, int64_t N, int64_t K,
-                        uint8_t* codes, uint8_t* scales);
+int skinny_unpack_nvfp4(const void* w_packed, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales);
 
 /* Bytes of the packed FP8 buffer for an N x K weight; 0 if N <= 0, K <= 0 or
  * K % 16 != 0. */
@@ -133,11 +131,10 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
 int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
 
 /* NVFP4 weight-only GEMM: y = x . W^T with W from skinny_pack_nvfp4.
- *   x            device [M][K] FP16, 16-byte aligned.
+ *   x            device [M][K] FP16, 16-byte aligned, read-only during the call.
  *   M            1..8 (rows of x: tokens of one decode / verify round).
  *   K            multiple of 16.
- *   w_packed     device, packed codes, 16-byte aligned.
- *   w_scales     device, packed UE4M3 scales, 16-byte aligned.
+ *   w_packed     device, from skinny_pack_nvfp4 (codes and block scales), 16-byte aligned.
  *   global_scale FP32 per-tensor scale, applied to the FP32 sum.
  *   N            output features.
  *   y            device [M][N], FP16 (RNE) or FP32 per out_dtype, 4-byte aligned.
@@ -150,9 +147,8 @@ int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
  * summation order differs from exact arithmetic, and it is fixed, so results
  * are bitwise reproducible run to run for a given shape and device.
  * Errors: see skinny_status. */
-int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_packed, const void* w_scales,
-                      float global_scale, int64_t N, void* y, int out_dtype, void* workspace,
-                      size_t workspace_bytes, void* stream);
+int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_packed, float global_scale, int64_t N,
+                      void* y, int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /* FP8 (E4M3) weight-only GEMM with a per-output-channel FP32 scale.
  *   w_packed       device, from skinny_pack_fp8, 16-byte aligned.
@@ -186,8 +182,8 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
  * share the one array, so calls that can overlap on the GPU (different
  * streams, or concurrent graph branches) race and corrupt each other's
  * results: serialise them. */
-int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, const void* w_packed, const void* w_scales,
-                                float global_scale, int64_t N, void* y, int out_dtype, void* stream);
+int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
+                                int64_t N, void* y, int out_dtype, void* stream);
 
 /* Size in bytes of the static scratch array used by skinny_nvfp4_gemm_static_ws. */
 size_t skinny_static_workspace_capacity(void);

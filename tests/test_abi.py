@@ -54,9 +54,9 @@ ALIGNED = 1 << 20  # a fake, 16-byte aligned address: never dereferenced by thes
     (dict(ws=ALIGNED + 8), sk.ERR_ALIGNMENT),
 ])
 def test_nvfp4_argument_checks(kw, status):
-    a = dict(x=ALIGNED, M=1, K=64, w=ALIGNED, s=ALIGNED, N=32, y=ALIGNED, out=0, ws=None)
+    a = dict(x=ALIGNED, M=1, K=64, w=ALIGNED, N=32, y=ALIGNED, out=0, ws=None)
     a.update(kw)
-    st = sk.library().skinny_nvfp4_gemm(a["x"], a["M"], a["K"], a["w"], a["s"], 1.0, a["N"], a["y"], a["out"],
+    st = sk.library().skinny_nvfp4_gemm(a["x"], a["M"], a["K"], a["w"], 1.0, a["N"], a["y"], a["out"],
                                         a["ws"], 0, None)
     assert st == status
 

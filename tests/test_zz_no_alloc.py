@@ -29,8 +29,8 @@ DEV = "cuda"
 def _call_static(x, w, y):
     out = sk.OUT_F32 if y.dtype == torch.float32 else sk.OUT_F16
     st = sk.library().skinny_nvfp4_gemm_static_ws(
-        x.data_ptr(), x.shape[0], w.K, w.codes.data_ptr(), w.scales.data_ptr(), ctypes.c_float(w.global_scale),
-        w.N, y.data_ptr(), out, torch.cuda.current_stream().cuda_stream)
+        x.data_ptr(), x.shape[0], w.K, w.data.data_ptr(), ctypes.c_float(w.global_scale), w.N, y.data_ptr(), out,
+        torch.cuda.current_stream().cuda_stream)
     assert st == sk.OK, sk.status_string(st)
 
 
@@ -62,6 +62,6 @@ def test_static_workspace_rejects_oversized_shape():
     assert cap == 4 << 20
     # More 256-row tiles than the counters region can hold after the partials.
     n_big = 1 << 30
-    st = sk.library().skinny_nvfp4_gemm_static_ws(1 << 20, 1, 16, 1 << 20, 1 << 20, ctypes.c_float(1.0), n_big,
-                                                  1 << 20, sk.OUT_F32, None)
+    st = sk.library().skinny_nvfp4_gemm_static_ws(1 << 20, 1, 16, 1 << 20, ctypes.c_float(1.0), n_big, 1 << 20,
+                                                  sk.OUT_F32, None)
     assert st == sk.ERR_UNSUPPORTED
