@@ -1,14 +1,13 @@
 // layout.h -- the packed weight layout shared by the host packer and the
 // sm_100a kernels (private to libskinny; the public ABI only sees byte counts).
 //
-// Tiles.  W[N][K] is cut into tiles of 256 output rows x 128 columns, stored in
+// Tiles.  W[N][K] is cut into tiles of 256 output rows x 256 columns, stored in
 // the order tile(g, c) = g * C + c (g = row tile, c = K tile), so a CTA that
-// walks a contiguous range of tiles streams one contiguous byte range, and
-// consecutive tiles can be fetched together by one bulk copy.  An NVFP4 tile
-// is 16384 code bytes followed by its 2048 UE4M3 scale bytes (18432 bytes);
-// an FP8 tile is 32768 bytes.
+// walks a contiguous range of tiles streams one contiguous byte range, one
+// bulk copy per tile.  An NVFP4 tile is 32768 code bytes followed by its 4096
+// UE4M3 scale bytes (36864 bytes); an FP8 tile is 65536 bytes.
 //
-// Inside a tile: 16 strips of 16 rows; each strip has two 64-column chunks.
+// Inside a tile: 16 strips of 16 rows; each strip has four 64-column chunks.
 // One chunk of one strip is laid out for a warp-wide sequence of four
 // m16n8k16 tensor-core steps j = 0..3: lane l = 4*gid + t owns rows
 // {gid, gid+8} of the strip and the 16 logical columns [16t, 16t+16) of the
@@ -31,13 +30,16 @@ constexpr int kTileRows = 256;       // output rows per tile
 constexpr int kStripRows = 16;       // rows per MMA strip (the m16 of m16n8k16)
 constexpr int kStrips = kTileRows / kStripRows;
 constexpr int kChunkK = 64;          // K per strip chunk (four k16 steps)
-constexpr int kTileK = 128;          // K per tile: two chunks
+constexpr int kTileK = 256;          // K per tile: four chunks
 constexpr int kChunks = kTileK / kChunkK;
 
-constexpr int kNvfp4TileCodeBytes = kTileRows * kTileK / 2;       // 16384
-constexpr int kNvfp4TileScaleBytes = kTileRows * kTileK / 16;     // 2048
+constexpr int kNvfp4TileCodeBytes = kTileRows * kTileK / 2;       // 32768
+constexpr int kNvfp4TileScaleBytes = kTileRows * kTileK / 16;     // 4096
 constexpr int kNvfp4TileBytes = kNvfp4TileCodeBytes + kNvfp4TileScaleBytes;
-constexpr int kFp8TileBytes = kTileRows * kTileK;                 // 32768
+constexpr int kFp8TileBytes = kTileRows * kTileK;                 // 65536
+constexpr int kNvfp4StripCodeBytes = kChunks * 512;   // one strip: 4 chunks x 32 lanes x 16 bytes
+constexpr int kNvfp4StripScaleBytes = kChunks * 64;   // one strip: 4 chunks x 64 scale bytes
+constexpr int kFp8StripBytes = kChunks * 1024;        // one strip: 4 chunks x 32 lanes x 32 bytes
 
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
@@ -60,7 +62,7 @@ inline Slot tile_slot(int r, int k)
     s.j = j;
     s.reg = h + 2 * (o / 2);
     s.e = o % 2;
-    s.word = strip * (kChunks * 512) + ch * 512 + (4 * gid + t) * 16 + 4 * j;  // NVFP4 placement
+    s.word = strip * kNvfp4StripCodeBytes + ch * 512 + (4 * gid + t) * 16 + 4 * j;  // NVFP4 placement
     return s;
 }
 
@@ -72,8 +74,8 @@ inline uint32_t nvfp4_put(uint32_t word, const Slot& s, uint32_t code)
 
 inline uint32_t nvfp4_get(uint32_t word, const Slot& s) { return (word >> (8 * s.reg + 4 * s.e)) & 0xFu; }
 
-// Byte offset, inside the 2048 scale bytes of an NVFP4 tile, of the UE4M3 scale of row
-// r (0..255) and 16-column block b (0..7).  A lane reads its two scales (rows
+// Byte offset, inside the 4096 scale bytes of an NVFP4 tile, of the UE4M3 scale of
+// row r (0..255) and 16-column block b (0..15).  A lane reads its two scales (rows
 // gid and gid+8 of its strip, block t of the chunk) as one 16-bit word: row
 // gid in the low byte (cvt.rn.f16x2.e4m3x2 turns the low byte into the low
 // half).
@@ -82,10 +84,10 @@ inline int nvfp4_scale_offset(int r, int b)
     const int strip = r / 16, rr = r % 16;
     const int gid = rr % 8, h = rr / 8;
     const int ch = b / 4, t = b % 4;
-    return strip * 128 + ch * 64 + t * 16 + gid * 2 + h;
+    return strip * kNvfp4StripScaleBytes + ch * 64 + t * 16 + gid * 2 + h;
 }
 
-// Byte offset, inside a 32768-byte FP8 tile, of element (row r, column k).
+// Byte offset, inside a 65536-byte FP8 tile, of element (row r, column k).
 // A lane's 32 bytes per chunk: step j in bytes 8j..8j+7, register r in bytes
 // 2r, 2r+1, element e in byte e (cvt.rn.f16x2.e4m3x2 turns the low byte into
 // the low half).
@@ -95,7 +97,7 @@ inline int fp8_offset(int r, int k)
     const int strip = r / 16, rr = r % 16;
     const int gid = rr % 8;
     const int ch = k / 64, t = (k % 64) / 16;
-    return strip * (kChunks * 1024) + ch * 1024 + (4 * gid + t) * 32 + 8 * s.j + 2 * s.reg + s.e;
+    return strip * kFp8StripBytes + ch * 1024 + (4 * gid + t) * 32 + 8 * s.j + 2 * s.reg + s.e;
 }
 
 }  // namespace skinny

@@ -7,12 +7,14 @@
 // their way out of HBM and become FP16 in registers for the tensor cores;
 // M=8 is the k=7 speculative-verify round).  The design here is B200-first:
 //
-//  * One persistent CTA per SM: 16 consumer warps + 1 producer warp.  The
-//    producer streams 256-row x 128-column weight tiles (16 KB NVFP4 codes +
-//    2 KB block scales, or 32 KB FP8) and the matching slice of x with bulk
-//    copies (the TMA engine, cp.async.bulk) into a shared-memory ring of 8
-//    (NVFP4) or 6 (FP8) stages guarded by mbarriers, so well over 100 KB per
-//    SM is in flight without spending registers on it.
+//  * One persistent CTA per SM with 16 warps.  Weights stream in 256-row x
+//    128-column tiles (16 KB NVFP4 codes + 2 KB block scales, or 32 KB FP8),
+//    two consecutive tiles per ring stage, each stage ONE bulk copy (the TMA
+//    engine, cp.async.bulk): a bulk copy costs its issuing thread ~150 ns, so
+//    copies must be large.  Stages are guarded by mbarriers; the warp that is
+//    last to release a slot issues its refill (no producer warp).
+//  * Activations are read by each lane straight from x (L1-cached), one stage
+//    ahead of use; they are tiny and shared by all CTAs.
 //  * Weights are decoded with Blackwell's native converts: one
 //    cvt.rn.f16x2.e2m1x2 per two FP4 codes (exact), the UE4M3 block scale
 //    with cvt.rn.f16x2.e4m3x2 and one f16x2 multiply (exact: e2m1 * ue4m3 has
@@ -41,12 +43,15 @@
 
 namespace skinny {
 
-// 16 consumer warps + 1 producer warp.  Consumer warp w handles strips
-// 2*(w%8) and 2*(w%8)+1 of every tile, in K chunk w/8; warps w and w+8 thus
-// hold the two K halves of the same 32 rows and add them at flush time.
+// 16 warps, all consumers.  Warp w handles strips 2*(w%8) and 2*(w%8)+1 of
+// every tile, in K chunk w/8; warps w and w+8 thus hold the two K halves of
+// the same 32 rows and add them at flush time.  There is no producer warp:
+// thread 0 issues the first stages, and each later stage is issued by the
+// warp that is last to release the ring slot it refills (so 16 warps keep
+// 4 warps per SM sub-partition and up to 128 registers each).
 constexpr int kConsumerWarps = 16;
 constexpr int kPairs = kConsumerWarps / 2;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kThreads = kConsumerWarps * 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 constexpr int kMaxDevices = 64;
 
@@ -60,14 +65,13 @@ __device__ unsigned int g_device_error;
 template <int FMT>
 struct Tile;
 
-// One ring stage holds kUnits consecutive tiles, fetched by ONE bulk copy:
-// every cp.async.bulk costs its issuing thread on the order of 150 ns on
-// B200, so copies must be large (>= 32 KB) to stream HBM at full rate.
+// One ring stage holds one 256 x 256 tile, fetched by ONE bulk copy (36 KB
+// NVFP4, 64 KB FP8): every cp.async.bulk costs its issuing thread on the
+// order of 150 ns on B200, so copies must be large to stream HBM at full rate.
 template <>
 struct Tile<SKINNY_FMT_NVFP4> {
-    static constexpr int kBytes = kNvfp4TileBytes;        // 16 KB codes + 2 KB scales
+    static constexpr int kBytes = kNvfp4TileBytes;        // 32 KB codes + 4 KB scales
     static constexpr int kScalesOff = kNvfp4TileCodeBytes;
-    static constexpr int kUnits = 2;
     static constexpr int kStages = 5;
 };
 
@@ -75,21 +79,22 @@ template <>
 struct Tile<SKINNY_FMT_FP8> {
     static constexpr int kBytes = kFp8TileBytes;
     static constexpr int kScalesOff = 0;
-    static constexpr int kUnits = 2;
     static constexpr int kStages = 3;
 };
 
-// Shared memory: kStages ring stages of kUnits tiles, then the flush exchange
+// Shared memory: kStages ring stages (one tile each), then the flush exchange
 // buffer (two parities of 8 pairs x 2 strips x 32 lanes x float4), then the
-// mbarriers.
+// mbarriers, the per-slot release counters and the flush ticket flag.
 template <int FMT>
 struct Smem {
     static constexpr int kStages = Tile<FMT>::kStages;
-    static constexpr int kStageBytes = Tile<FMT>::kUnits * Tile<FMT>::kBytes;
+    static constexpr int kStageBytes = Tile<FMT>::kBytes;
     static constexpr int kXchgOff = kStages * kStageBytes;
     static constexpr int kXchgBytes = 2 * kPairs * 2 * 32 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
-    static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
+    static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
+    static constexpr int kFlagOff = kCountOff + kStages * 4;       // int last_flag
+    static constexpr int kBytes = kFlagOff + 16;
     static_assert(kStageBytes % 16 == 0, "stage alignment");
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
@@ -224,30 +229,13 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int slot
     }
 }
 
+// Issue unit q of this CTA (one tile, one bulk copy) into ring slot s.
 template <int FMT>
-__device__ void produce(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int u_begin,
-                        int n_units)
+__device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int q, int u_begin)
 {
-    using S = Smem<FMT>;
-    constexpr int kStages = S::kStages, kUnits = Tile<FMT>::kUnits;
-    const uint64_t pol_w = ptx::policy_evict_first();
-    const int n_stages = (n_units + kUnits - 1) / kUnits;
-    int issued = 0;
-    for (int q = 0; q < n_stages; ++q) {
-        const int s = q % kStages;
-        if (q >= kStages && !ptx::mbar_wait(&empty[s], ((q / kStages) & 1) ^ 1, kWaitLimitNs)) {
-            atomicOr(&g_device_error, 2u);
-            break;
-        }
-        const int u0 = u_begin + q * kUnits;
-        const uint32_t bytes = (uint32_t)min(kUnits, n_units - q * kUnits) * Tile<FMT>::kBytes;
-        ptx::mbar_arrive_expect_tx(&full[s], bytes);
-        ptx::bulk_g2s(smem + s * S::kStageBytes, p.codes + (size_t)u0 * Tile<FMT>::kBytes, bytes, &full[s], pol_w);
-        issued = q + 1;
-    }
-    // No bulk copy may still be landing in this CTA's shared memory at exit.
-    for (int q = max(0, issued - kStages); q < issued; ++q)
-        if (!ptx::mbar_wait(&full[q % kStages], (q / kStages) & 1, kWaitLimitNs)) atomicOr(&g_device_error, 4u);
+    ptx::mbar_arrive_expect_tx(&full[s], Tile<FMT>::kBytes);
+    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, p.codes + (size_t)(u_begin + q) * Tile<FMT>::kBytes,
+                  Tile<FMT>::kBytes, &full[s], ptx::policy_evict_first());
 }
 
 // The B fragments of one K tile for this lane: token gid (row xrow of x),
@@ -266,19 +254,16 @@ __device__ __forceinline__ void load_b(const uint16_t* xrow, bool valid, int kb,
     bx[4] = x1.x; bx[5] = x1.y; bx[6] = x1.z; bx[7] = x1.w;
 }
 
-// Per-warp state of the consumer loop.  A warp owns strips 2*pair and
-// 2*pair+1 of every tile in K chunk ch, and keeps one accumulator per strip and
-// per unit parity (the two tiles of a stage are processed together, so four
-// independent MMA chains hide the tensor-core latency); the parities are added
-// in a fixed order when a row tile is flushed.
+// Per-warp state of the consumer loop.  A warp owns strips 2*pair, 2*pair+1
+// and K chunks 2*half, 2*half+1 of every tile: four strip chunks, each with
+// its own accumulator chain (hiding the tensor-core latency); the two chunk
+// accumulators of a strip are added in a fixed order when a row tile is
+// flushed.
 template <int FMT>
 struct Consumer {
-    float acc[2][2][4];     // [unit parity][strip][fragment]
-    uint32_t lane_codes;    // this lane's code bytes of strip 2*pair, chunk ch, inside a tile
-    uint32_t lane_scale;    // this lane's scale word of strip 2*pair, chunk ch (NVFP4)
-    const uint16_t* xrow;   // x row of token gid
-    bool xvalid;            // gid < M
-    int K;
+    float acc[2][2][4];     // [chunk parity][strip][fragment]
+    uint32_t lane_codes;    // this lane's code bytes of strip 2*pair, chunk 2*half, inside a tile
+    uint32_t lane_scale;    // this lane's scale word of strip 2*pair, chunk 2*half (NVFP4)
 
     __device__ __forceinline__ void zero()
     {
@@ -290,7 +275,7 @@ struct Consumer {
                 for (int r = 0; r < 4; ++r) acc[u][q][r] = 0.f;
     }
 
-    // The per-strip sums of both parities (fixed order).
+    // The per-strip sums of both chunks (fixed order).
     __device__ __forceinline__ void total(float (&tot)[2][4]) const
     {
 #pragma unroll
@@ -299,31 +284,33 @@ struct Consumer {
             for (int r = 0; r < 4; ++r) tot[q][r] = acc[0][q][r] + acc[1][q][r];
     }
 
-    // NU (1 or 2) consecutive units of one row tile, tiles at shared addresses
-    // tile[u], activations bx[u]: all shared loads first, then the decode and
-    // MMAs of the NU x 2 strip chunks interleaved step by step.
-    template <int NU>
-    __device__ __forceinline__ void compute(const uint32_t (&tile)[2], const uint32_t (&bx)[2][8])
+    // The warp's four strip chunks of the tile at shared address `tile`;
+    // bx[u] holds the activations of chunk 2*half + u.  All shared loads are
+    // issued first, then the decode and MMA steps of the four chains
+    // interleave.
+    __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][8])
     {
         if constexpr (FMT == SKINNY_FMT_NVFP4) {
-            uint4 cw[NU][2];
-            uint32_t s0[NU][2], s8[NU][2];
+            uint4 cw[2][2];
+            uint32_t s0[2][2], s8[2][2];
 #pragma unroll
-            for (int u = 0; u < NU; ++u)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int q = 0; q < 2; ++q) cw[u][q] = ptx::lds128(tile[u] + lane_codes + q * 1024);
+                for (int q = 0; q < 2; ++q)
+                    cw[u][q] = ptx::lds128(tile + lane_codes + q * kNvfp4StripCodeBytes + u * 512);
 #pragma unroll
-            for (int u = 0; u < NU; ++u)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    const uint32_t sc = ptx::e4m3x2_to_f16x2(ptx::lds16(tile[u] + lane_scale + q * 128));
+                    const uint32_t sc =
+                        ptx::e4m3x2_to_f16x2(ptx::lds16(tile + lane_scale + q * kNvfp4StripScaleBytes + u * 64));
                     s0[u][q] = ptx::dup_lo(sc);   // scale of row gid
                     s8[u][q] = ptx::dup_hi(sc);   // scale of row gid+8
                 }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int u = 0; u < NU; ++u)
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         const uint32_t w = j == 0 ? cw[u][q].x : j == 1 ? cw[u][q].y : j == 2 ? cw[u][q].z : cw[u][q].w;
@@ -334,18 +321,19 @@ struct Consumer {
                         ptx::mma_f16_16816(acc[u][q], a, bx[u][2 * j], bx[u][2 * j + 1]);
                     }
         } else {
-            uint4 cw[NU][2][2];
+            uint4 cw[2][2][2];
 #pragma unroll
-            for (int u = 0; u < NU; ++u)
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    cw[u][q][0] = ptx::lds128(tile[u] + lane_codes + q * 2048);
-                    cw[u][q][1] = ptx::lds128(tile[u] + lane_codes + q * 2048 + 16);
+                    const uint32_t base = tile + lane_codes + q * kFp8StripBytes + u * 1024;
+                    cw[u][q][0] = ptx::lds128(base);
+                    cw[u][q][1] = ptx::lds128(base + 16);
                 }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int u = 0; u < NU; ++u)
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         const uint4& v = cw[u][q][j >> 1];
@@ -359,109 +347,107 @@ struct Consumer {
     }
 };
 
-// The unit coordinates (row tile g, K tile c) of unit u_begin + i.
-struct Cursor {
-    int g, c;
-    __device__ __forceinline__ void next(int C)
-    {
-        if (++c == C) {
-            c = 0;
-            ++g;
-        }
-    }
-};
-
 template <int FMT>
 __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, volatile int* last_flag,
                         int u_begin, int n_units, int b, int P, int UQ, int warp, int lane)
 {
     using S = Smem<FMT>;
-    constexpr int kStages = S::kStages, kUnits = Tile<FMT>::kUnits;
-    static_assert(kUnits == 2, "the consumer processes two tiles per stage");
-    constexpr int kTileBytes = Tile<FMT>::kBytes;
+    constexpr int kStages = S::kStages;
     const int gid = lane >> 2, t = lane & 3;
-    const int ch = warp / kPairs, pair = warp % kPairs;
-    const int kb_lane = ch * kChunkK + 16 * t;
+    const int half = warp / kPairs, pair = warp % kPairs;
 
     Consumer<FMT> w;
     w.zero();
     if constexpr (FMT == SKINNY_FMT_NVFP4) {
-        w.lane_codes = (2 * pair) * 1024 + ch * 512 + lane * 16;
-        w.lane_scale = Tile<FMT>::kScalesOff + (2 * pair) * 128 + ch * 64 + t * 16 + gid * 2;
+        w.lane_codes = (2 * pair) * kNvfp4StripCodeBytes + (2 * half) * 512 + lane * 16;
+        w.lane_scale = Tile<FMT>::kScalesOff + (2 * pair) * kNvfp4StripScaleBytes + (2 * half) * 64 + t * 16 + gid * 2;
     } else {
-        w.lane_codes = (2 * pair) * 2048 + ch * 1024 + lane * 32;
+        w.lane_codes = (2 * pair) * kFp8StripBytes + (2 * half) * 1024 + lane * 32;
         w.lane_scale = 0;
     }
-    w.xvalid = gid < p.M;
-    w.xrow = p.x + (size_t)(w.xvalid ? gid : 0) * p.K;
-    w.K = p.K;
+    // Activations: token gid, columns c*256 + (2*half + u)*64 + [16t, 16t+16).
+    const bool xvalid = gid < p.M;
+    const uint16_t* xrow = p.x + (size_t)(xvalid ? gid : 0) * p.K;
+    const int kb_lane = 2 * half * kChunkK + 16 * t;
 
     const int first_g = u_begin / p.C;
     int cur_g = first_g, parity = 0;
-    Cursor cu{first_g, u_begin - first_g * p.C};   // first unit of the stage being processed
+    int g = first_g, c = u_begin - first_g * p.C;   // tile being processed
+    int nc = c;                                      // K tile whose activations are fetched next
     const uint32_t smem32 = ptx::smem_addr(smem);
-    const int n_stages = (n_units + kUnits - 1) / kUnits;
+    int* released = reinterpret_cast<int*>(smem + S::kCountOff);
+
+    uint32_t bx[2][2][8];   // ping-pong: [buffer][chunk][words]
+    load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, bx[0][0]);
+    load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, bx[0][1]);
 
     bool ok = true;
     int s = 0;
     uint32_t phase = 0;
-    for (int q = 0; q < n_stages; ++q) {
-        const int n_here = min(kUnits, n_units - q * kUnits);
-        Cursor c1 = cu;
-        c1.next(p.C);
-        // Activations of this stage's units (L1/L2 hits; in flight during the wait below).
-        uint32_t bx[2][8];
-        load_b(w.xrow, w.xvalid, cu.c * kTileK + kb_lane, p.K, bx[0]);
-        if (n_here > 1) load_b(w.xrow, w.xvalid, c1.c * kTileK + kb_lane, p.K, bx[1]);
-
+    // One tile per iteration; the body is written for buffer B = i & 1 (the
+    // loop is unrolled by two so the ping-pong buffers stay in registers).
+    auto step = [&](int i, uint32_t (&cur)[2][8], uint32_t (&nxt)[2][8]) {
+        if (++nc == p.C) nc = 0;
+        if (i + 1 < n_units) {   // next tile's activations, one tile ahead
+            load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, nxt[0]);
+            load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, nxt[1]);
+        }
         if (ok) {
             // All lanes agree on the outcome, so the warp stays converged.
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[s], phase, kWaitLimitNs));
             if (!ok && lane == 0) atomicOr(&g_device_error, 1u);
         }
-        const uint32_t tiles[2] = {smem32 + s * S::kStageBytes, smem32 + s * S::kStageBytes + kTileBytes};
-        // unit 0 of the stage
-        if (cu.g != cur_g) {
+        if (g != cur_g) {
             float tot[2][4];
             w.total(tot);
             flush<FMT>(p, tot, cur_g, cur_g == first_g ? 0 : 1, parity, smem, last_flag, b, P, UQ, warp, lane);
             parity ^= 1;
             w.zero();
-            cur_g = cu.g;
+            cur_g = g;
         }
-        if (n_here == 2 && c1.g == cur_g) {
-            if (ok) w.template compute<2>(tiles, bx);                 // both units, one row tile
-        } else {
-            if (ok) w.template compute<1>(tiles, bx);                 // unit 0 alone
-            if (n_here == 2) {                                        // unit 1 starts a new row tile
-                float tot[2][4];
-                w.total(tot);
-                flush<FMT>(p, tot, cur_g, cur_g == first_g ? 0 : 1, parity, smem, last_flag, b, P, UQ, warp, lane);
-                parity ^= 1;
-                w.zero();
-                cur_g = c1.g;
-                const uint32_t t1[2] = {tiles[1], tiles[1]};
-                uint32_t b1[2][8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) b1[0][k] = b1[1][k] = bx[1][k];
-                if (ok) w.template compute<1>(t1, b1);
-            }
-        }
-        cu = c1;
-        cu.next(p.C);
         if (ok) {
+            w.compute(smem32 + s * S::kStageBytes, cur);
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&empty[s]);
+            if (lane == 0) {
+                // Release the slot; the last of the 16 warps to do so refills it.
+                ptx::mbar_arrive(&empty[s]);
+                if (atomicAdd(&released[s], 1) == kConsumerWarps - 1) {
+                    released[s] = 0;
+                    if (i + kStages < n_units) {
+                        if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
+                            issue_stage<FMT>(p, smem, full, s, i + kStages, u_begin);
+                        else
+                            atomicOr(&g_device_error, 2u);
+                    }
+                }
+            }
         }
         if (++s == kStages) {
             s = 0;
             phase ^= 1;
         }
+        if (++c == p.C) {
+            c = 0;
+            ++g;
+        }
+    };
+    int i = 0;
+    for (; i + 1 < n_units; i += 2) {
+        step(i, bx[0], bx[1]);
+        step(i + 1, bx[1], bx[0]);
     }
+    if (i < n_units) step(i, bx[0], bx[1]);
+
     if (n_units > 0) {
         float tot[2][4];
         w.total(tot);
         flush<FMT>(p, tot, cur_g, cur_g == first_g ? 0 : 1, parity, smem, last_flag, b, P, UQ, warp, lane);
+    }
+    if (!ok && threadIdx.x == 0) {
+        // After a wait gave up, tiles may still be landing in shared memory:
+        // wait (bounded) for the last ring's worth before the CTA exits.
+        for (int q = max(0, n_units - kStages); q < n_units; ++q)
+            if (!ptx::mbar_wait(&full[q % kStages], (q / kStages) & 1, kWaitLimitNs)) atomicOr(&g_device_error, 4u);
     }
 }
 
@@ -472,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
     uint64_t* empty = full + S::kStages;
-    volatile int* last_flag = reinterpret_cast<volatile int*>(empty + S::kStages);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + S::kFlagOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, b = blockIdx.x;
@@ -484,15 +470,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         for (int s = 0; s < S::kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], kConsumerWarps);
+            reinterpret_cast<int*>(smem + S::kCountOff)[s] = 0;
         }
         ptx::fence_mbar_init();
+        for (int q = 0; q < S::kStages && q < n_units; ++q) issue_stage<FMT>(p, smem, full, q, q, u_begin);
     }
     __syncthreads();
 
-    if (warp == kConsumerWarps) {
-        if (lane == 0) produce<FMT>(p, smem, full, empty, u_begin, n_units);
-        return;
-    }
     consume<FMT>(p, smem, full, empty, last_flag, u_begin, n_units, b, P, UQ, warp, lane);
 }
 

@@ -73,11 +73,11 @@ int skinny_version(void);
  * Host-side layout routines (pure CPU, no CUDA call).
  *
  * The kernels read W in a private tiled order: tiles of 256 output rows x
- * 128 columns, consecutive in memory along K then N, so that a run of tiles is
+ * 256 columns, consecutive in memory along K then N, so that a run of tiles is
  * one contiguous bulk copy and each lane of a warp finds its tensor-core
  * operand bytes in one 16-byte word.  An NVFP4 tile carries its UE4M3 block
- * scales (16 KB codes + 2 KB scales); an FP8 tile is 32 KB.  Rows are padded
- * to a multiple of 256 and K to a multiple of 128 with zero codes and zero
+ * scales (32 KB codes + 4 KB scales); an FP8 tile is 64 KB.  Rows are padded
+ * to a multiple of 256 and K to a multiple of 256 with zero codes and zero
  * scales, which contribute nothing.  The caller packs once per weight and
  * copies the result to the device.
  * ---------------------------------------------------------------------- */
