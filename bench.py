@@ -66,6 +66,24 @@ def step_bytes() -> int:
     return sum(gemm_bytes(s, M) for M in PASSES for s in si.MIXED_LAYER)
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest `value` over all ranks (each rank times its own replica; the
+    job takes as long as the slowest one)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Aggregate effective GB/s of `world` replicas that each ran `steps` steps in `ms`."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -359,10 +377,14 @@ def cpu_baseline(target_s: float = 12.0):
     threads = oracle.default_threads()
     frac = oracle_sample_frac(target_s, threads)
     items = _oracle_inputs(frac)
-    t = _oracle_run(items, threads)
-    return {"value": round(_oracle_bytes(items) / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+    t, reps = 0.0, 0
+    while t < 0.8 * target_s or reps == 0:   # the whole workload may take less than target_s
+        t += _oracle_run(items, threads)
+        reps += 1
+    return {"value": round(reps * _oracle_bytes(items) / t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
             "sample": "float64 C oracle, %d threads, on the first %.3f%% of the rows of each of the 5 GEMMs of %s at "
-                      "M=1 and M=8 (same byte formula), %.1f s" % (threads, 100 * frac, WORKLOAD, t)}
+                      "M=1 and M=8 (same byte formula), %d pass(es), %.1f s" % (threads, 100 * frac, WORKLOAD, reps, t)}
 
 
 def reference_arm(args):
@@ -487,22 +509,15 @@ def main(argv=None):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert sk.device_error(clear=True) == 0, "a device-side wait gave up"
 
     e2e_ms, h2d, d2h = e2e_run(weights, xs, ys, ws, args.steps, args.warmup)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     sb = step_bytes()
-    value = world * sb * args.steps / (ms * 1e-3) / 1e9
-    e2e_value = world * sb * args.steps / (e2e_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, sb, args.steps, ms)
+    e2e_value = whole_job_gbs(world, sb, args.steps, e2e_ms)
 
     # Roofline of the dominant kernel (the NVFP4 GEMM: 8 of 10 launches, most of the bytes).
     per = []

@@ -1,13 +1,13 @@
 // layout.h -- the packed weight layout shared by the host packer and the
 // sm_100a kernels (private to libskinny; the public ABI only sees byte counts).
 //
-// Tiles.  W[N][K] is cut into tiles of 256 output rows x 256 columns, stored in
+// Tiles.  W[N][K] is cut into tiles of 128 output rows x 512 columns, stored in
 // the order tile(g, c) = g * C + c (g = row tile, c = K tile), so a CTA that
 // walks a contiguous range of tiles streams one contiguous byte range, one
 // bulk copy per tile.  An NVFP4 tile is 32768 code bytes followed by its 4096
 // UE4M3 scale bytes (36864 bytes); an FP8 tile is 65536 bytes.
 //
-// Inside a tile: 16 strips of 16 rows; each strip has four 64-column chunks.
+// Inside a tile: 8 strips of 16 rows; each strip has eight 64-column chunks.
 // One chunk of one strip is laid out for a warp-wide sequence of four
 // m16n8k16 tensor-core steps j = 0..3: lane l = 4*gid + t owns rows
 // {gid, gid+8} of the strip and the 16 logical columns [16t, 16t+16) of the
@@ -26,24 +26,24 @@
 
 namespace skinny {
 
-constexpr int kTileRows = 256;       // output rows per tile
+constexpr int kTileRows = 128;       // output rows per tile
 constexpr int kStripRows = 16;       // rows per MMA strip (the m16 of m16n8k16)
 constexpr int kStrips = kTileRows / kStripRows;
 constexpr int kChunkK = 64;          // K per strip chunk (four k16 steps)
-constexpr int kTileK = 256;          // K per tile: four chunks
+constexpr int kTileK = 512;          // K per tile: eight chunks
 constexpr int kChunks = kTileK / kChunkK;
 
 constexpr int kNvfp4TileCodeBytes = kTileRows * kTileK / 2;       // 32768
 constexpr int kNvfp4TileScaleBytes = kTileRows * kTileK / 16;     // 4096
 constexpr int kNvfp4TileBytes = kNvfp4TileCodeBytes + kNvfp4TileScaleBytes;
 constexpr int kFp8TileBytes = kTileRows * kTileK;                 // 65536
-constexpr int kNvfp4StripCodeBytes = kChunks * 512;   // one strip: 4 chunks x 32 lanes x 16 bytes
-constexpr int kNvfp4StripScaleBytes = kChunks * 64;   // one strip: 4 chunks x 64 scale bytes
-constexpr int kFp8StripBytes = kChunks * 1024;        // one strip: 4 chunks x 32 lanes x 32 bytes
+constexpr int kNvfp4StripCodeBytes = kChunks * 512;   // one strip: 8 chunks x 32 lanes x 16 bytes
+constexpr int kNvfp4StripScaleBytes = kChunks * 64;   // one strip: 8 chunks x 64 scale bytes
+constexpr int kFp8StripBytes = kChunks * 1024;        // one strip: 8 chunks x 32 lanes x 32 bytes
 
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
-// Where element (row r in 0..255, column k in 0..127) of a tile lives.
+// Where element (row r in 0..127, column k in 0..511) of a tile lives.
 struct Slot {
     int word;   // byte offset of its 32-bit word inside the tile's codes
     int j;      // MMA step (word index inside the lane's 16 / 32 bytes)
@@ -75,7 +75,7 @@ inline uint32_t nvfp4_put(uint32_t word, const Slot& s, uint32_t code)
 inline uint32_t nvfp4_get(uint32_t word, const Slot& s) { return (word >> (8 * s.reg + 4 * s.e)) & 0xFu; }
 
 // Byte offset, inside the 4096 scale bytes of an NVFP4 tile, of the UE4M3 scale of
-// row r (0..255) and 16-column block b (0..15).  A lane reads its two scales (rows
+// row r (0..127) and 16-column block b (0..31).  A lane reads its two scales (rows
 // gid and gid+8 of its strip, block t of the chunk) as one 16-bit word: row
 // gid in the low byte (cvt.rn.f16x2.e4m3x2 turns the low byte into the low
 // half).

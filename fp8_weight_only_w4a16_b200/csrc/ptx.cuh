@@ -168,6 +168,22 @@ __device__ __forceinline__ uint16_t lds16(uint32_t addr)
     return v;
 }
 
+// Programmatic dependent launch: let the next kernel in the stream start its
+// CTAs as ours retire, and wait for the previous kernel's memory before
+// touching anything it may have written.  Both are no-ops for a launch
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Ticket for the split-K fixup: release this CTA's partial sums (ordered
+// before it by the preceding CTA barrier) and acquire the other contributors'.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v)
+{
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -43,22 +43,24 @@
 
 namespace skinny {
 
-// 16 warps, all consumers.  Warp w handles strips 2*(w%8) and 2*(w%8)+1 of
-// every tile, in K chunk w/8; warps w and w+8 thus hold the two K halves of
-// the same 32 rows and add them at flush time.  There is no producer warp:
-// thread 0 issues the first stages, and each later stage is issued by the
-// warp that is last to release the ring slot it refills (so 16 warps keep
-// 4 warps per SM sub-partition and up to 128 registers each).
+// 16 warps, all consumers.  Warp w handles strip pair sp = w % 4 (strips
+// 2sp, 2sp+1) and chunk pair kq = w / 4 (chunks 2kq, 2kq+1) of every tile, so
+// warps sp, sp+4, sp+8, sp+12 hold the four K quarters of the same 32 rows
+// and add them at flush time.  There is no producer warp: thread 0 issues
+// the first stages, and each later stage is issued by the warp that is last
+// to release the ring slot it refills (so 16 warps keep 4 warps per SM
+// sub-partition and up to 128 registers each).
 constexpr int kConsumerWarps = 16;
-constexpr int kPairs = kConsumerWarps / 2;
+constexpr int kStripPairs = kStrips / 2;                       // 4
+constexpr int kChunkPairs = kConsumerWarps / kStripPairs;      // 4
 constexpr int kThreads = kConsumerWarps * 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 constexpr int kMaxDevices = 64;
 
-static_assert(kPairs * 2 == kStrips, "two strips per consumer warp");
+static_assert(kChunkPairs * 2 == kChunks, "two chunks per consumer warp");
 
-// Barrier ids: 0 = __syncthreads, 1 = the 16 consumer warps, 2 = warps 0..7.
-constexpr uint32_t kBarConsumers = 1, kBarLow = 2;
+// Named barrier id of the 16 consumer warps (0 is __syncthreads).
+constexpr uint32_t kBarConsumers = 1;
 
 __device__ unsigned int g_device_error;
 
@@ -83,14 +85,14 @@ struct Tile<SKINNY_FMT_FP8> {
 };
 
 // Shared memory: kStages ring stages (one tile each), then the flush exchange
-// buffer (two parities of 8 pairs x 2 strips x 32 lanes x float4), then the
+// buffer (two parities of 16 warps x 2 strips x 32 lanes x float4), then the
 // mbarriers, the per-slot release counters and the flush ticket flag.
 template <int FMT>
 struct Smem {
     static constexpr int kStages = Tile<FMT>::kStages;
     static constexpr int kStageBytes = Tile<FMT>::kBytes;
     static constexpr int kXchgOff = kStages * kStageBytes;
-    static constexpr int kXchgBytes = 2 * kPairs * 2 * 32 * 16;
+    static constexpr int kXchgBytes = 2 * kConsumerWarps * 2 * 32 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
     static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
     static constexpr int kFlagOff = kCountOff + kStages * 4;       // int last_flag
@@ -105,7 +107,7 @@ struct Params {
     const float* channel_scale;   // FP8 per-channel scale [N]
     void* y;                      // [M][N]
     int* counters;                // [G] arrival tickets (split-K only)
-    float4* partials;             // [P][2][8 pairs][2 strips][32 lanes] (split-K only)
+    float2* partials;             // [P][2][16 warps][32 lanes] (split-K only)
     float out_scale;              // NVFP4 per-tensor scale (FP8: unused, the channel scales apply)
     int M, K, N;
     int C;                        // K tiles per row tile
@@ -126,105 +128,93 @@ __device__ __forceinline__ int owner_of(int u, int P, int UQ, int Q)
     return (int)((((int64_t)(u / Q) + 1) * P - 1) / UQ);
 }
 
-__device__ __forceinline__ int partial_index(int cta, int slot, int pair, int lane)
+// Partial sums of one contribution: [cta][slot][16 warps][32 lanes] float2.
+__device__ __forceinline__ int partial_index(int cta, int slot, int warp, int lane)
 {
-    return ((cta * 2 + slot) * kPairs + pair) * 64 + lane;  // + 32 for the pair's second strip
+    return ((cta * 2 + slot) * kConsumerWarps + warp) * 32 + lane;
 }
 
+// One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
+// tokens 2t and 2t+1 of this lane (v[0], v[1]).
 template <int FMT>
-__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2][4], int g, int pair, int lane)
+__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane)
 {
     const int gid = lane >> 2, t = lane & 3;
+    const int n = g * kTileRows + strip * kStripRows + gid + 8 * h;
+    if (n >= p.N) return;
+    const float sc = (FMT == SKINNY_FMT_NVFP4) ? p.out_scale : p.channel_scale[n];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int n = g * kTileRows + (2 * pair + q) * kStripRows + gid + 8 * h;
-            if (n >= p.N) continue;
-            const float sc = (FMT == SKINNY_FMT_NVFP4) ? p.out_scale : p.channel_scale[n];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int m = 2 * t + e;
-                if (m >= p.M) continue;
-                const float val = v[q][2 * h + e] * sc;
-                const size_t idx = (size_t)m * p.N + n;
-                if (p.out_f32)
-                    static_cast<float*>(p.y)[idx] = val;
-                else
-                    static_cast<__half*>(p.y)[idx] = __float2half_rn(val);
-            }
-        }
+    for (int e = 0; e < 2; ++e) {
+        const int m = 2 * t + e;
+        if (m >= p.M) continue;
+        const float val = v[e] * sc;
+        const size_t idx = (size_t)m * p.N + n;
+        if (p.out_f32)
+            static_cast<float*>(p.y)[idx] = val;
+        else
+            static_cast<__half*>(p.y)[idx] = __float2half_rn(val);
     }
 }
 
-// Finish row tile g.  Warps 8..15 hand their K half to warps 0..7 (which add
-// chunk 0 + chunk 1, a fixed order).  If this CTA covered the whole K range
-// of g, warps 0..7 write y; otherwise they publish the partial sums, take a
-// ticket, and the last contributor adds all partials in CTA order.
+// Finish row tile g.  The four warps of a strip pair (sp, sp+4, sp+8, sp+12)
+// hold the four K quarters of strips 2sp and 2sp+1; through shared memory each
+// of them takes one quarter of the strip pair's outputs (strip 2sp + kq/2,
+// rows gid + 8*(kq%2)) and adds the four K quarters in order (a fixed order).
+// If this CTA covered the whole K range of g, every warp writes its slice of
+// y; otherwise the warps publish their partial sums, take a ticket, and the
+// CTA that arrives last adds all contributors' partials in CTA order (all 16
+// warps, loads batched so the L2 round trips overlap).
 template <int FMT>
 __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int slot, int parity, uint8_t* smem,
                       volatile int* last_flag, int b, int P, int UQ, int warp, int lane)
 {
-    float4* xchg = reinterpret_cast<float4*>(smem + Smem<FMT>::kXchgOff) + parity * (kPairs * 64);
-    const int pair = warp & (kPairs - 1);
-    if (warp >= kPairs) {
-        xchg[pair * 64 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-        xchg[pair * 64 + 32 + lane] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-    }
+    float4* xchg = reinterpret_cast<float4*>(smem + Smem<FMT>::kXchgOff) + parity * (kConsumerWarps * 64);
+    const int sp = warp % kStripPairs, kq = warp / kStripPairs;
+    const int sq = kq >> 1, h = kq & 1;          // this warp finishes strip 2sp+sq, rows gid+8h
+    xchg[warp * 64 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+    xchg[warp * 64 + 32 + lane] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    if (warp >= kPairs) return;
-
-    float tot[2][4];
-    {
-        const float4 h0 = xchg[pair * 64 + lane], h1 = xchg[pair * 64 + 32 + lane];
-        tot[0][0] = acc[0][0] + h0.x; tot[0][1] = acc[0][1] + h0.y; tot[0][2] = acc[0][2] + h0.z; tot[0][3] = acc[0][3] + h0.w;
-        tot[1][0] = acc[1][0] + h1.x; tot[1][1] = acc[1][1] + h1.y; tot[1][2] = acc[1][2] + h1.z; tot[1][3] = acc[1][3] + h1.w;
+    float tot[2] = {0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < kChunkPairs; ++k) {
+        const float4 v = xchg[(k * kStripPairs + sp) * 64 + sq * 32 + lane];
+        tot[0] += h ? v.z : v.x;
+        tot[1] += h ? v.w : v.y;
     }
+    const int strip = 2 * sp + sq;
     const int c_first = owner_of(g * p.C, P, UQ, p.Q);
     const int c_last = owner_of(g * p.C + p.C - 1, P, UQ, p.Q);
     if (c_first == c_last) {
-        epilogue<FMT>(p, tot, g, pair, lane);
+        epilogue<FMT>(p, tot, g, strip, h, lane);
         return;
     }
-    float4* mine = p.partials + partial_index(b, slot, pair, lane);
-    mine[0] = make_float4(tot[0][0], tot[0][1], tot[0][2], tot[0][3]);
-    mine[32] = make_float4(tot[1][0], tot[1][1], tot[1][2], tot[1][3]);
-    ptx::named_barrier_sync(kBarLow, kPairs * 32);
-    if (threadIdx.x == 0) {
-        __threadfence();  // release: the CTA's partials (ordered before by the barrier)
-        const int old = atomicAdd(&p.counters[g], 1);
-        __threadfence();  // acquire: the other contributors' partials
-        *last_flag = (old == c_last - c_first);
-    }
-    ptx::named_barrier_sync(kBarLow, kPairs * 32);
+    p.partials[partial_index(b, slot, warp, lane)] = make_float2(tot[0], tot[1]);
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
+    if (threadIdx.x == 0) *last_flag = (ptx::atomic_add_acq_rel_gpu(&p.counters[g], 1) == c_last - c_first);
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
     if (*last_flag) {
-        // Add the contributors' partials in CTA order; their loads are issued in
-        // batches of kBatch so that the L2 round trips overlap.
-        constexpr int kBatch = 2;
-        float sum[2][4] = {};
+        constexpr int kBatch = 8;
+        float sum[2] = {0.f, 0.f};
         for (int c0 = c_first; c0 <= c_last; c0 += kBatch) {
-            float4 v[kBatch][2];
+            float2 v[kBatch];
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
                 const int cc = c0 + k;
                 if (cc <= c_last && cc != b) {
                     const int sl = (g == range_start(cc, P, UQ, p.Q) / p.C) ? 0 : 1;
-                    const float4* src = p.partials + partial_index(cc, sl, pair, lane);
-                    v[k][0] = __ldcg(src);
-                    v[k][1] = __ldcg(src + 32);
+                    v[k] = __ldcg(p.partials + partial_index(cc, sl, warp, lane));
                 } else {
-                    v[k][0] = make_float4(tot[0][0], tot[0][1], tot[0][2], tot[0][3]);
-                    v[k][1] = make_float4(tot[1][0], tot[1][1], tot[1][2], tot[1][3]);
+                    v[k] = make_float2(tot[0], tot[1]);
                 }
             }
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
                 if (c0 + k > c_last) break;
-                sum[0][0] += v[k][0].x; sum[0][1] += v[k][0].y; sum[0][2] += v[k][0].z; sum[0][3] += v[k][0].w;
-                sum[1][0] += v[k][1].x; sum[1][1] += v[k][1].y; sum[1][2] += v[k][1].z; sum[1][3] += v[k][1].w;
+                sum[0] += v[k].x;
+                sum[1] += v[k].y;
             }
         }
-        epilogue<FMT>(p, sum, g, pair, lane);
+        epilogue<FMT>(p, sum, g, strip, h, lane);
         if (threadIdx.x == 0) p.counters[g] = 0;  // ready for the next call
     }
 }
@@ -254,16 +244,16 @@ __device__ __forceinline__ void load_b(const uint16_t* xrow, bool valid, int kb,
     bx[4] = x1.x; bx[5] = x1.y; bx[6] = x1.z; bx[7] = x1.w;
 }
 
-// Per-warp state of the consumer loop.  A warp owns strips 2*pair, 2*pair+1
-// and K chunks 2*half, 2*half+1 of every tile: four strip chunks, each with
+// Per-warp state of the consumer loop.  A warp owns strips 2sp, 2sp+1 and K
+// chunks 2kq, 2kq+1 of every tile: four strip chunks, each with
 // its own accumulator chain (hiding the tensor-core latency); the two chunk
 // accumulators of a strip are added in a fixed order when a row tile is
 // flushed.
 template <int FMT>
 struct Consumer {
     float acc[2][2][4];     // [chunk parity][strip][fragment]
-    uint32_t lane_codes;    // this lane's code bytes of strip 2*pair, chunk 2*half, inside a tile
-    uint32_t lane_scale;    // this lane's scale word of strip 2*pair, chunk 2*half (NVFP4)
+    uint32_t lane_codes;    // this lane's code bytes of strip 2sp, chunk 2kq, inside a tile
+    uint32_t lane_scale;    // this lane's scale word of strip 2sp, chunk 2kq (NVFP4)
 
     __device__ __forceinline__ void zero()
     {
@@ -285,7 +275,7 @@ struct Consumer {
     }
 
     // The warp's four strip chunks of the tile at shared address `tile`;
-    // bx[u] holds the activations of chunk 2*half + u.  All shared loads are
+    // bx[u] holds the activations of chunk 2kq + u.  All shared loads are
     // issued first, then the decode and MMA steps of the four chains
     // interleave.
     __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][8])
@@ -354,21 +344,21 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     using S = Smem<FMT>;
     constexpr int kStages = S::kStages;
     const int gid = lane >> 2, t = lane & 3;
-    const int half = warp / kPairs, pair = warp % kPairs;
+    const int sp = warp % kStripPairs, kq = warp / kStripPairs;
 
     Consumer<FMT> w;
     w.zero();
     if constexpr (FMT == SKINNY_FMT_NVFP4) {
-        w.lane_codes = (2 * pair) * kNvfp4StripCodeBytes + (2 * half) * 512 + lane * 16;
-        w.lane_scale = Tile<FMT>::kScalesOff + (2 * pair) * kNvfp4StripScaleBytes + (2 * half) * 64 + t * 16 + gid * 2;
+        w.lane_codes = (2 * sp) * kNvfp4StripCodeBytes + (2 * kq) * 512 + lane * 16;
+        w.lane_scale = Tile<FMT>::kScalesOff + (2 * sp) * kNvfp4StripScaleBytes + (2 * kq) * 64 + t * 16 + gid * 2;
     } else {
-        w.lane_codes = (2 * pair) * kFp8StripBytes + (2 * half) * 1024 + lane * 32;
+        w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 32;
         w.lane_scale = 0;
     }
-    // Activations: token gid, columns c*256 + (2*half + u)*64 + [16t, 16t+16).
+    // Activations: token gid, columns c*512 + (2kq + u)*64 + [16t, 16t+16).
     const bool xvalid = gid < p.M;
     const uint16_t* xrow = p.x + (size_t)(xvalid ? gid : 0) * p.K;
-    const int kb_lane = 2 * half * kChunkK + 16 * t;
+    const int kb_lane = 2 * kq * kChunkK + 16 * t;
 
     const int first_g = u_begin / p.C;
     int cur_g = first_g, parity = 0;
@@ -467,15 +457,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int n_units = range_start(b + 1, P, UQ, p.Q) - u_begin;
 
     if (threadIdx.x == 0) {
+        ptx::pdl_launch_dependents();
         for (int s = 0; s < S::kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], kConsumerWarps);
             reinterpret_cast<int*>(smem + S::kCountOff)[s] = 0;
         }
         ptx::fence_mbar_init();
+        // The packed weights are read-only parameters: start streaming them
+        // before the previous kernel in the stream has finished.
         for (int q = 0; q < S::kStages && q < n_units; ++q) issue_stage<FMT>(p, smem, full, q, q, u_begin);
     }
     __syncthreads();
+    // x, y, the channel scales and the workspace may belong to the previous
+    // kernel: touch them only once it has completed.
+    ptx::pdl_wait_prior_grid();
 
     consume<FMT>(p, smem, full, empty, last_flag, u_begin, n_units, b, P, UQ, warp, lane);
 }
@@ -535,7 +531,7 @@ static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* p
     pl->U = (int)(G * C);
     const int UQ = split ? pl->U : pl->G;
     pl->P = UQ < sms ? UQ : sms;
-    pl->partial_bytes = (size_t)sms * 2 * kPairs * 64 * sizeof(float4);
+    pl->partial_bytes = (size_t)sms * 2 * kConsumerWarps * 32 * sizeof(float2);
     pl->workspace_bytes = pl->partial_bytes + ((size_t)G * sizeof(int) + 255) / 256 * 256;
     return SKINNY_OK;
 }
@@ -568,9 +564,21 @@ static int launch(Params p, int64_t N, int64_t K, void* workspace, size_t worksp
     p.C = pl.C;
     p.U = pl.U;
     p.Q = split ? 1 : pl.C;
-    p.partials = split ? static_cast<float4*>(workspace) : nullptr;
+    p.partials = split ? static_cast<float2*>(workspace) : nullptr;
     p.counters = split ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes) : nullptr;
-    gemm_kernel<FMT><<<pl.P, kThreads, Smem<FMT>::kBytes, stream>>>(p);
+    // Programmatic dependent launch: the kernel may start (and prefetch its
+    // weights) while the previous kernel in the stream is finishing.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Smem<FMT>::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT>, p) != cudaSuccess) return SKINNY_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SKINNY_OK : SKINNY_ERR_CUDA;
 }
 

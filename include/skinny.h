@@ -37,6 +37,13 @@
  *     default stream).  Their status covers the argument checks and the
  *     launch only; a fault inside a kernel appears on the stream as usual and
  *     a device-side wait that gave up is reported by skinny_device_error().
+ *   - GEMM kernels are launched with programmatic dependent launch: one may
+ *     begin while the previous kernel in the stream is still running, and
+ *     starts reading the packed weights (and nothing else) before that
+ *     kernel completes.  The packed weights must therefore not be written by
+ *     the kernel launched just before the GEMM on the same stream; x, y, the
+ *     FP8 channel scales and the workspace are touched only after it
+ *     completes.  (Weights are model parameters: packed once, then read.)
  */
 #ifndef SKINNY_H
 #define SKINNY_H
@@ -72,12 +79,12 @@ int skinny_version(void);
 /* ------------------------------------------------------------------------
  * Host-side layout routines (pure CPU, no CUDA call).
  *
- * The kernels read W in a private tiled order: tiles of 256 output rows x
- * 256 columns, consecutive in memory along K then N, so that a run of tiles is
+ * The kernels read W in a private tiled order: tiles of 128 output rows x
+ * 512 columns, consecutive in memory along K then N, so that a run of tiles is
  * one contiguous bulk copy and each lane of a warp finds its tensor-core
  * operand bytes in one 16-byte word.  An NVFP4 tile carries its UE4M3 block
  * scales (32 KB codes + 4 KB scales); an FP8 tile is 64 KB.  Rows are padded
- * to a multiple of 256 and K to a multiple of 256 with zero codes and zero
+ * to a multiple of 128 and K to a multiple of 512 with zero codes and zero
  * scales, which contribute nothing.  The caller packs once per weight and
  * copies the result to the device.
  * ---------------------------------------------------------------------- */
@@ -119,9 +126,9 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
 /* Size of the optional split-K workspace for one GEMM of this format and
  * shape on the CURRENT device (it depends on the SM count).  A workspace lets
  * the kernel split K across CTAs so that every SM streams the same number of
- * weight bytes (a short-N shape such as 5120 x 5120 has too few 256-row tiles
+ * weight bytes (a short-N shape such as 5120 x 5120 has too few 128-row tiles
  * to fill 148 SMs otherwise).  It holds FP32 partial sums followed by one
- * arrival counter per 256-row tile; the counters must be ZERO before the
+ * arrival counter per 128-row tile; the counters must be ZERO before the
  * first use and every completed call leaves them zero again, so zero-fill the
  * workspace once (cudaMemset) and reuse it.  Its layout is the same for every
  * shape on a device, so a workspace sized for the largest call serves calls of
@@ -173,7 +180,7 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
  * bytes (4 MiB) that every GPU which loads this library holds until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
  * allocating library routine.  Shapes whose scratch would not fit (more than
- * about 442k 256-row tiles on a 148-SM B200) return SKINNY_ERR_UNSUPPORTED.
+ * about 745k 128-row tiles on a 148-SM B200) return SKINNY_ERR_UNSUPPORTED.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, which may load the library's device code); make that

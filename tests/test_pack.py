@@ -11,7 +11,7 @@ def test_nvfp4_roundtrip(N, K):
     codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     scales = rng.integers(0, 0x7F, size=(N, K // 16), dtype=np.uint8)
     pc = sk.pack_nvfp4(codes, scales)
-    Np, Kp = -(-N // 256) * 256, -(-K // 256) * 256
+    Np, Kp = -(-N // 128) * 128, -(-K // 512) * 512
     assert pc.size == Np * Kp // 2 + Np * Kp // 16
     c2, s2 = sk.unpack_nvfp4(pc, N, K)
     assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
@@ -26,17 +26,17 @@ def test_fp8_roundtrip(N, K):
     q = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
     q[(q & 0x7F) == 0x7F] = 0x11
     pc = sk.pack_fp8(q)
-    assert pc.size == (-(-N // 256) * 256) * (-(-K // 256) * 256)
+    assert pc.size == (-(-N // 128) * 128) * (-(-K // 512) * 512)
     assert np.array_equal(sk.unpack_fp8(pc, N, K), q)
     assert np.count_nonzero(pc) == np.count_nonzero(q)
 
 
 def test_nvfp4_element_lands_in_its_tile():
-    """A single nonzero code at (n, k) lands in tile (n // 256) * C + k // 256, in
+    """A single nonzero code at (n, k) lands in tile (n // 128) * C + k // 512, in
     the strip of row n, the 64-column chunk of k, and the 16-byte word of lane
     4*((n%16)%8) + (k%64)//16 (all its bits inside one 32-bit word)."""
-    N, K = 600, 768
-    C = K // 256
+    N, K = 300, 1536
+    C = K // 512
     rng = np.random.default_rng(0)
     for _ in range(200):
         n, k = int(rng.integers(N)), int(rng.integers(K))
@@ -46,11 +46,11 @@ def test_nvfp4_element_lands_in_its_tile():
         idx = np.nonzero(pc)[0]
         assert idx.size >= 1 and idx[-1] // 4 == idx[0] // 4
         tile, off = divmod(int(idx[0]), 36864)
-        assert tile == (n // 256) * C + k // 256
-        strip, rem = divmod(off, 2048)
-        assert strip == (n % 256) // 16
+        assert tile == (n // 128) * C + k // 512
+        strip, rem = divmod(off, 4096)
+        assert strip == (n % 128) // 16
         chunk, rem = divmod(rem, 512)
-        assert chunk == (k % 256) // 64
+        assert chunk == (k % 512) // 64
         assert rem // 16 == 4 * ((n % 16) % 8) + (k % 64) // 16
 
 
@@ -79,7 +79,7 @@ def test_nvfp4_lane_words_decode_to_their_slots():
     16-bit scale word: row gid in the low byte, row gid+8 in the high byte."""
     import ml_dtypes
 
-    N, K = 256, 256
+    N, K = 128, 512
     rng = np.random.default_rng(5)
     codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     pc = sk.pack_nvfp4(codes, np.zeros((N, K // 16), np.uint8))
@@ -87,11 +87,11 @@ def test_nvfp4_lane_words_decode_to_their_slots():
     nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(N, K)
     val = nib.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
     words = pc.view(np.uint32)
-    for strip in range(16):
-        for chunk in range(4):
+    for strip in range(8):
+        for chunk in range(8):
             for lane in range(32):
                 gid, t = lane // 4, lane % 4
-                base = (strip * 2048 + chunk * 512 + lane * 16) // 4
+                base = (strip * 4096 + chunk * 512 + lane * 16) // 4
                 dec = _emulate_lane_decode(words[base:base + 4])
                 i = 0
                 for j in range(4):
@@ -105,30 +105,30 @@ def test_nvfp4_lane_words_decode_to_their_slots():
 
 
 def test_nvfp4_lane_scale_words():
-    N, K = 256, 256
+    N, K = 128, 512
     rng = np.random.default_rng(7)
     scales = rng.integers(0, 0x7F, size=(N, K // 16), dtype=np.uint8)
     pc = sk.pack_nvfp4(np.zeros((N, K // 2), np.uint8), scales)
     sc = pc[32768:]
-    for strip in range(16):
-        for chunk in range(4):
+    for strip in range(8):
+        for chunk in range(8):
             for lane in range(32):
                 gid, t = lane // 4, lane % 4
-                off = strip * 256 + chunk * 64 + t * 16 + gid * 2
+                off = strip * 512 + chunk * 64 + t * 16 + gid * 2
                 assert sc[off] == scales[strip * 16 + gid, chunk * 4 + t]
                 assert sc[off + 1] == scales[strip * 16 + gid + 8, chunk * 4 + t]
 
 
 def test_fp8_lane_bytes_hold_their_slots():
-    N, K = 256, 256
+    N, K = 128, 512
     rng = np.random.default_rng(6)
     q = rng.integers(0, 0x7F, size=(N, K), dtype=np.uint8)
     pc = sk.pack_fp8(q)
-    for strip in range(16):
-        for chunk in range(4):
+    for strip in range(8):
+        for chunk in range(8):
             for lane in range(32):
                 gid, t = lane // 4, lane % 4
-                base = strip * 4096 + chunk * 1024 + lane * 32
+                base = strip * 8192 + chunk * 1024 + lane * 32
                 for j in range(4):
                     for r in range(4):
                         for e in range(2):
