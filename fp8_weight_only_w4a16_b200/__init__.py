@@ -205,7 +205,7 @@ def workspace_bytes(fmt: int, M: int, N: int, K: int) -> int:
 
 
 def make_workspace(fmt: int, M: int, N: int, K: int, device="cuda"):
-    """A zero-filled workspace (its arrival counters must start at zero)."""
+    """A zero-filled workspace (its partial-sum slots must start at zero)."""
     import torch
 
     return torch.zeros(workspace_bytes(fmt, M, N, K), dtype=torch.uint8, device=device)

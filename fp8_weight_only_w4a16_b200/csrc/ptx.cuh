@@ -175,13 +175,20 @@ __device__ __forceinline__ uint16_t lds16(uint32_t addr)
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Ticket for the split-K fixup: release this CTA's partial sums (ordered
-// before it by the preceding CTA barrier) and acquire the other contributors'.
-__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v)
+// Split-K partial sums travel between CTAs through global memory with
+// volatile (relaxed, system-scope) accesses: the finisher polls a slot until
+// the publisher's value appears, so neither side may use a weak access that
+// could be cached in L1 or merged away.
+__device__ __forceinline__ void st_volatile_v2(uint2* p, uint2 v)
 {
-    int old;
-    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+    asm volatile("st.volatile.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+__device__ __forceinline__ uint2 ld_volatile_v2(const uint2* p)
+{
+    uint2 v;
+    asm volatile("ld.volatile.global.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads)

@@ -7,13 +7,16 @@
 // their way out of HBM and become FP16 in registers for the tensor cores;
 // M=8 is the k=7 speculative-verify round).  The design here is B200-first:
 //
-//  * One persistent CTA per SM with 16 warps.  Weights stream in 256-row x
-//    128-column tiles (16 KB NVFP4 codes + 2 KB block scales, or 32 KB FP8),
-//    two consecutive tiles per ring stage, each stage ONE bulk copy (the TMA
-//    engine, cp.async.bulk): a bulk copy costs its issuing thread ~150 ns, so
-//    copies must be large.  Stages are guarded by mbarriers; the warp that is
-//    last to release a slot issues its refill (no producer warp).
-//  * Activations are read by each lane straight from x (L1-cached), one stage
+//  * One persistent CTA per SM with 16 warps.  Weights stream in 128-row x
+//    512-column tiles (32 KB NVFP4 codes + 4 KB block scales, or 64 KB FP8),
+//    one tile per ring stage, each stage ONE bulk copy (the TMA engine,
+//    cp.async.bulk): a bulk copy costs its issuing thread ~150 ns, so copies
+//    must be large.  Stages are guarded by mbarriers; the warp that is last
+//    to release a slot issues its refill (no producer warp).
+//  * Programmatic dependent launch: a CTA starts streaming its first tiles
+//    while the previous kernel in the stream is still finishing, and touches
+//    x, y and the workspace only after that kernel has completed.
+//  * Activations are read by each lane straight from x (L1-cached), one tile
 //    ahead of use; they are tiny and shared by all CTAs.
 //  * Weights are decoded with Blackwell's native converts: one
 //    cvt.rn.f16x2.e2m1x2 per two FP4 codes (exact), the UE4M3 block scale
@@ -23,13 +26,18 @@
 //  * m16n8k16 tensor-core MMAs with FP32 accumulation; the MMA's n = 8
 //    columns are the M <= 8 tokens.  The tensor rate this needs (16 flop per
 //    weight) is a small fraction of the SM's, so tensor cores are never the
-//    bound.  Warps w and w+8 take the two 64-column halves of a tile for the
-//    same 32 rows and add their sums (in a fixed order) when a tile is done.
+//    bound.
 //  * Work is balanced by "stream-K": the grid's CTAs take equal contiguous
-//    ranges of the tile sequence.  A 256-row tile whose K range is split
-//    between CTAs is finished by the last CTA to arrive (an atomic ticket, no
-//    spinning), which adds the FP32 partials in CTA order -- so results are
-//    bitwise reproducible.  Without a workspace, CTAs take whole row tiles.
+//    ranges of the tile sequence and walk them BACKWARDS.  A row tile whose
+//    K range is split between CTAs is then finished by its highest-numbered
+//    contributor, which reaches it at the end of its range, while every other
+//    contributor reached it at the start of its own (or holds nothing else).
+//    Contributors publish their FP32 partial sums with plain stores, encoded
+//    so that an all-zero word means "not written yet"; the finisher polls for
+//    them (bounded), adds them in CTA order -- results are bitwise
+//    reproducible -- and zeroes the slots again.  No atomics, no fences, and
+//    each CTA publishes at most once.  Without a workspace, CTAs take whole
+//    row tiles.
 //  * Every wait is bounded (1 s of global time); a wait that gives up sets a
 //    bit in g_device_error and its CTA winds down instead of hanging.
 #include <cuda_fp16.h>
@@ -62,12 +70,18 @@ static_assert(kChunkPairs * 2 == kChunks, "two chunks per consumer warp");
 // Named barrier id of the 16 consumer warps (0 is __syncthreads).
 constexpr uint32_t kBarConsumers = 1;
 
+// Bits of g_device_error: which bounded wait gave up.
+constexpr unsigned kErrFullWait = 1u;      // a warp waiting for a tile
+constexpr unsigned kErrEmptyWait = 2u;     // the refilling warp waiting for a slot
+constexpr unsigned kErrDrainWait = 4u;     // draining copies in flight after an abort
+constexpr unsigned kErrPartialWait = 8u;   // a finisher waiting for a partial sum
+
 __device__ unsigned int g_device_error;
 
 template <int FMT>
 struct Tile;
 
-// One ring stage holds one 256 x 256 tile, fetched by ONE bulk copy (36 KB
+// One ring stage holds one 128 x 512 tile, fetched by ONE bulk copy (36 KB
 // NVFP4, 64 KB FP8): every cp.async.bulk costs its issuing thread on the
 // order of 150 ns on B200, so copies must be large to stream HBM at full rate.
 template <>
@@ -86,7 +100,7 @@ struct Tile<SKINNY_FMT_FP8> {
 
 // Shared memory: kStages ring stages (one tile each), then the flush exchange
 // buffer (two parities of 16 warps x 2 strips x 32 lanes x float4), then the
-// mbarriers, the per-slot release counters and the flush ticket flag.
+// mbarriers and the per-slot release counters.
 template <int FMT>
 struct Smem {
     static constexpr int kStages = Tile<FMT>::kStages;
@@ -95,8 +109,7 @@ struct Smem {
     static constexpr int kXchgBytes = 2 * kConsumerWarps * 2 * 32 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
     static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
-    static constexpr int kFlagOff = kCountOff + kStages * 4;       // int last_flag
-    static constexpr int kBytes = kFlagOff + 16;
+    static constexpr int kBytes = kCountOff + kStages * 4;
     static_assert(kStageBytes % 16 == 0, "stage alignment");
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
@@ -104,10 +117,9 @@ struct Smem {
 struct Params {
     const uint16_t* x;            // [M][K] fp16 bits
     const uint8_t* codes;         // packed tiles (NVFP4 tiles carry their block scales)
-    const float* channel_scale;   // FP8 per-channel scale [N]
+    const float* channel_scale;   // FP8 per-output-channel scale [N]
     void* y;                      // [M][N]
-    int* counters;                // [G] arrival tickets (split-K only)
-    float2* partials;             // [P][2][16 warps][32 lanes] (split-K only)
+    uint2* partials;              // [P][16 warps][32 lanes] encoded float pairs (split-K only)
     float out_scale;              // NVFP4 per-tensor scale (FP8: unused, the channel scales apply)
     int M, K, N;
     int C;                        // K tiles per row tile
@@ -123,16 +135,46 @@ __host__ __device__ __forceinline__ int range_start(int b, int P, int UQ, int Q)
 }
 
 // The CTA whose range holds tile u (inverse of range_start).
-__device__ __forceinline__ int owner_of(int u, int P, int UQ, int Q)
+__host__ __device__ __forceinline__ int owner_of(int u, int P, int UQ, int Q)
 {
     return (int)((((int64_t)(u / Q) + 1) * P - 1) / UQ);
 }
 
-// Partial sums of one contribution: [cta][slot][16 warps][32 lanes] float2.
-__device__ __forceinline__ int partial_index(int cta, int slot, int warp, int lane)
+// This CTA's range and the contributors of the row tiles at its two ends
+// (every row tile strictly inside the range is this CTA's alone).
+struct Sched {
+    int b;
+    int u_last;       // last tile of the range (processed first)
+    int n_units;
+    int first_g, last_g;
+    int first_owner;  // lowest contributor of row tile first_g
+    int last_owner;   // highest contributor of row tile last_g
+};
+
+__device__ __forceinline__ Sched make_sched(const Params& p, int b, int P)
 {
-    return ((cta * 2 + slot) * kConsumerWarps + warp) * 32 + lane;
+    const int UQ = p.U / p.Q;
+    Sched s;
+    s.b = b;
+    const int u_begin = range_start(b, P, UQ, p.Q);
+    s.n_units = range_start(b + 1, P, UQ, p.Q) - u_begin;
+    s.u_last = u_begin + s.n_units - 1;
+    s.first_g = u_begin / p.C;
+    s.last_g = s.u_last / p.C;
+    s.first_owner = owner_of(s.first_g * p.C, P, UQ, p.Q);
+    s.last_owner = owner_of(s.last_g * p.C + p.C - 1, P, UQ, p.Q);
+    return s;
 }
+
+// A published partial sum never encodes to zero: NaNs are made canonical
+// (0x7FC00000), so the one float pattern whose complement is zero
+// (0xFFFFFFFF, a NaN) never occurs.  A zeroed slot therefore reads "empty".
+__device__ __forceinline__ uint32_t encode_partial(float v)
+{
+    return ~(v == v ? __float_as_uint(v) : 0x7FC00000u);
+}
+
+__device__ __forceinline__ float decode_partial(uint32_t e) { return __uint_as_float(~e); }
 
 // One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
 // tokens 2t and 2t+1 of this lane (v[0], v[1]).
@@ -156,17 +198,19 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
     }
 }
 
-// Finish row tile g.  The four warps of a strip pair (sp, sp+4, sp+8, sp+12)
-// hold the four K quarters of strips 2sp and 2sp+1; through shared memory each
-// of them takes one quarter of the strip pair's outputs (strip 2sp + kq/2,
-// rows gid + 8*(kq%2)) and adds the four K quarters in order (a fixed order).
-// If this CTA covered the whole K range of g, every warp writes its slice of
-// y; otherwise the warps publish their partial sums, take a ticket, and the
-// CTA that arrives last adds all contributors' partials in CTA order (all 16
-// warps, loads batched so the L2 round trips overlap).
+// Finish (or contribute to) row tile g, whose K range CTAs c_first..c_last
+// share.  The four warps of a strip pair (sp, sp+4, sp+8, sp+12) hold the
+// four K quarters of strips 2sp and 2sp+1; through shared memory each of them
+// takes one quarter of the strip pair's outputs (strip 2sp + kq/2, rows
+// gid + 8*(kq%2)) and adds the four K quarters in order (a fixed order).
+//  * c_first == c_last: this CTA covered all of K; write y.
+//  * this CTA is not c_last: publish the partial sums in this CTA's slot.
+//  * this CTA is c_last (the finisher): wait for the slots of c_first ..
+//    c_last-1, add them in CTA order and then its own sums, write y, and
+//    zero the slots for the next call.
 template <int FMT>
-__device__ void flush(const Params& p, const float (&acc)[2][4], int g, int slot, int parity, uint8_t* smem,
-                      volatile int* last_flag, int b, int P, int UQ, int warp, int lane)
+__device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_first, int c_last, int parity,
+                      uint8_t* smem, int b, int warp, int lane)
 {
     float4* xchg = reinterpret_cast<float4*>(smem + Smem<FMT>::kXchgOff) + parity * (kConsumerWarps * 64);
     const int sp = warp % kStripPairs, kq = warp / kStripPairs;
@@ -182,50 +226,64 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int slot
         tot[1] += h ? v.w : v.y;
     }
     const int strip = 2 * sp + sq;
-    const int c_first = owner_of(g * p.C, P, UQ, p.Q);
-    const int c_last = owner_of(g * p.C + p.C - 1, P, UQ, p.Q);
     if (c_first == c_last) {
         epilogue<FMT>(p, tot, g, strip, h, lane);
         return;
     }
-    p.partials[partial_index(b, slot, warp, lane)] = make_float2(tot[0], tot[1]);
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    if (threadIdx.x == 0) *last_flag = (ptx::atomic_add_acq_rel_gpu(&p.counters[g], 1) == c_last - c_first);
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    if (*last_flag) {
-        constexpr int kBatch = 8;
-        float sum[2] = {0.f, 0.f};
-        for (int c0 = c_first; c0 <= c_last; c0 += kBatch) {
-            float2 v[kBatch];
+    if (b != c_last) {
+        ptx::st_volatile_v2(p.partials + (b * kConsumerWarps + warp) * 32 + lane,
+                            make_uint2(encode_partial(tot[0]), encode_partial(tot[1])));
+        return;
+    }
+    // Finisher.  The other contributors are lower-numbered CTAs; all but the
+    // middle ones (whose whole range lies in g) published long ago.
+    constexpr int kBatch = 8;
+    float sum[2] = {0.f, 0.f};
+    bool timed_out = false;
+    uint64_t t0 = 0;
+    for (int c0 = c_first; c0 < c_last; c0 += kBatch) {
+        uint2 v[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k)
+            v[k] = (c0 + k < c_last) ? ptx::ld_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane)
+                                     : make_uint2(1u, 1u);
+        for (uint32_t it = 0;; ++it) {
+            bool missing = false;
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
-                const int cc = c0 + k;
-                if (cc <= c_last && cc != b) {
-                    const int sl = (g == range_start(cc, P, UQ, p.Q) / p.C) ? 0 : 1;
-                    v[k] = __ldcg(p.partials + partial_index(cc, sl, warp, lane));
-                } else {
-                    v[k] = make_float2(tot[0], tot[1]);
+                if (v[k].x == 0u || v[k].y == 0u) {
+                    missing = true;
+                    v[k] = ptx::ld_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane);
                 }
             }
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                if (c0 + k > c_last) break;
-                sum[0] += v[k].x;
-                sum[1] += v[k].y;
+            if (!missing || timed_out) break;
+            if (it == 0) t0 = ptx::globaltimer_ns();
+            else if ((it & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                timed_out = true;
+                atomicOr(&g_device_error, kErrPartialWait);
             }
         }
-        epilogue<FMT>(p, sum, g, strip, h, lane);
-        if (threadIdx.x == 0) p.counters[g] = 0;  // ready for the next call
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            if (c0 + k < c_last) {
+                sum[0] += decode_partial(v[k].x);
+                sum[1] += decode_partial(v[k].y);
+                ptx::st_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane, make_uint2(0u, 0u));
+            }
+        }
     }
+    sum[0] += tot[0];
+    sum[1] += tot[1];
+    epilogue<FMT>(p, sum, g, strip, h, lane);
 }
 
-// Issue unit q of this CTA (one tile, one bulk copy) into ring slot s.
+// Put tile `u` into ring slot s with one bulk copy.
 template <int FMT>
-__device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int q, int u_begin)
+__device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int u)
 {
     ptx::mbar_arrive_expect_tx(&full[s], Tile<FMT>::kBytes);
-    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, p.codes + (size_t)(u_begin + q) * Tile<FMT>::kBytes,
-                  Tile<FMT>::kBytes, &full[s], ptx::policy_evict_first());
+    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, p.codes + (size_t)u * Tile<FMT>::kBytes, Tile<FMT>::kBytes,
+                  &full[s], ptx::policy_evict_first());
 }
 
 // The B fragments of one K tile for this lane: token gid (row xrow of x),
@@ -338,13 +396,14 @@ struct Consumer {
 };
 
 template <int FMT>
-__device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, volatile int* last_flag,
-                        int u_begin, int n_units, int b, int P, int UQ, int warp, int lane)
+__device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, const Sched& sc, int warp,
+                        int lane)
 {
     using S = Smem<FMT>;
     constexpr int kStages = S::kStages;
     const int gid = lane >> 2, t = lane & 3;
     const int sp = warp % kStripPairs, kq = warp / kStripPairs;
+    const int n_units = sc.n_units;
 
     Consumer<FMT> w;
     w.zero();
@@ -360,12 +419,21 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     const uint16_t* xrow = p.x + (size_t)(xvalid ? gid : 0) * p.K;
     const int kb_lane = 2 * kq * kChunkK + 16 * t;
 
-    const int first_g = u_begin / p.C;
-    int cur_g = first_g, parity = 0;
-    int g = first_g, c = u_begin - first_g * p.C;   // tile being processed
-    int nc = c;                                      // K tile whose activations are fetched next
+    // The range is walked from its last tile down to its first.
+    int cur_g = sc.last_g, parity = 0;
+    int g = sc.last_g, c = sc.u_last - sc.last_g * p.C;   // tile being processed
+    int nc = c;                                            // K tile whose activations are fetched next
     const uint32_t smem32 = ptx::smem_addr(smem);
     int* released = reinterpret_cast<int*>(smem + S::kCountOff);
+    // Contributors of a row tile: only the two at the ends of the range are shared.
+    auto flush_g = [&](int fg) {
+        float tot[2][4];
+        w.total(tot);
+        const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
+        const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
+        flush<FMT>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane);
+        parity ^= 1;
+    };
 
     uint32_t bx[2][2][8];   // ping-pong: [buffer][chunk][words]
     load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, bx[0][0]);
@@ -377,7 +445,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     // One tile per iteration; the body is written for buffer B = i & 1 (the
     // loop is unrolled by two so the ping-pong buffers stay in registers).
     auto step = [&](int i, uint32_t (&cur)[2][8], uint32_t (&nxt)[2][8]) {
-        if (++nc == p.C) nc = 0;
+        nc = (nc == 0 ? p.C : nc) - 1;
         if (i + 1 < n_units) {   // next tile's activations, one tile ahead
             load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, nxt[0]);
             load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, nxt[1]);
@@ -385,13 +453,10 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         if (ok) {
             // All lanes agree on the outcome, so the warp stays converged.
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[s], phase, kWaitLimitNs));
-            if (!ok && lane == 0) atomicOr(&g_device_error, 1u);
+            if (!ok && lane == 0) atomicOr(&g_device_error, kErrFullWait);
         }
         if (g != cur_g) {
-            float tot[2][4];
-            w.total(tot);
-            flush<FMT>(p, tot, cur_g, cur_g == first_g ? 0 : 1, parity, smem, last_flag, b, P, UQ, warp, lane);
-            parity ^= 1;
+            flush_g(cur_g);
             w.zero();
             cur_g = g;
         }
@@ -405,9 +470,9 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
                     released[s] = 0;
                     if (i + kStages < n_units) {
                         if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
-                            issue_stage<FMT>(p, smem, full, s, i + kStages, u_begin);
+                            issue_stage<FMT>(p, smem, full, s, sc.u_last - (i + kStages));
                         else
-                            atomicOr(&g_device_error, 2u);
+                            atomicOr(&g_device_error, kErrEmptyWait);
                     }
                 }
             }
@@ -416,10 +481,11 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
             s = 0;
             phase ^= 1;
         }
-        if (++c == p.C) {
-            c = 0;
-            ++g;
+        if (c == 0) {
+            c = p.C;
+            --g;
         }
+        --c;
     };
     int i = 0;
     for (; i + 1 < n_units; i += 2) {
@@ -428,16 +494,13 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
     if (i < n_units) step(i, bx[0], bx[1]);
 
-    if (n_units > 0) {
-        float tot[2][4];
-        w.total(tot);
-        flush<FMT>(p, tot, cur_g, cur_g == first_g ? 0 : 1, parity, smem, last_flag, b, P, UQ, warp, lane);
-    }
+    if (n_units > 0) flush_g(cur_g);
     if (!ok && threadIdx.x == 0) {
         // After a wait gave up, tiles may still be landing in shared memory:
         // wait (bounded) for the last ring's worth before the CTA exits.
         for (int q = max(0, n_units - kStages); q < n_units; ++q)
-            if (!ptx::mbar_wait(&full[q % kStages], (q / kStages) & 1, kWaitLimitNs)) atomicOr(&g_device_error, 4u);
+            if (!ptx::mbar_wait(&full[q % kStages], (q / kStages) & 1, kWaitLimitNs))
+                atomicOr(&g_device_error, kErrDrainWait);
     }
 }
 
@@ -448,13 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
     uint64_t* empty = full + S::kStages;
-    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + S::kFlagOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int P = gridDim.x, b = blockIdx.x;
-    const int UQ = p.U / p.Q;
-    const int u_begin = range_start(b, P, UQ, p.Q);
-    const int n_units = range_start(b + 1, P, UQ, p.Q) - u_begin;
+    const Sched sc = make_sched(p, blockIdx.x, gridDim.x);
 
     if (threadIdx.x == 0) {
         ptx::pdl_launch_dependents();
@@ -466,14 +525,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         ptx::fence_mbar_init();
         // The packed weights are read-only parameters: start streaming them
         // before the previous kernel in the stream has finished.
-        for (int q = 0; q < S::kStages && q < n_units; ++q) issue_stage<FMT>(p, smem, full, q, q, u_begin);
+        for (int q = 0; q < S::kStages && q < sc.n_units; ++q) issue_stage<FMT>(p, smem, full, q, sc.u_last - q);
     }
     __syncthreads();
     // x, y, the channel scales and the workspace may belong to the previous
     // kernel: touch them only once it has completed.
     ptx::pdl_wait_prior_grid();
 
-    consume<FMT>(p, smem, full, empty, last_flag, u_begin, n_units, b, P, UQ, warp, lane);
+    consume<FMT>(p, smem, full, empty, sc, warp, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -513,11 +572,11 @@ static int current_device(int* sms)
 }
 
 // Workspace layout (identical for every shape on a device, so one workspace
-// can serve calls of different shapes in turn): the partial-sum slots of up
-// to one CTA per SM first, then one arrival counter per row tile.
+// can serve calls of different shapes in turn): one partial-sum slot of
+// 16 warps x 32 lanes x 2 floats per CTA, for up to one CTA per SM.
 struct Plan {
     int G, C, U, P;
-    size_t partial_bytes, workspace_bytes;
+    size_t workspace_bytes;
 };
 
 static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* pl)
@@ -531,8 +590,7 @@ static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* p
     pl->U = (int)(G * C);
     const int UQ = split ? pl->U : pl->G;
     pl->P = UQ < sms ? UQ : sms;
-    pl->partial_bytes = (size_t)sms * 2 * kConsumerWarps * 32 * sizeof(float2);
-    pl->workspace_bytes = pl->partial_bytes + ((size_t)G * sizeof(int) + 255) / 256 * 256;
+    pl->workspace_bytes = (size_t)sms * kConsumerWarps * 32 * sizeof(uint2);
     return SKINNY_OK;
 }
 
@@ -564,8 +622,7 @@ static int launch(Params p, int64_t N, int64_t K, void* workspace, size_t worksp
     p.C = pl.C;
     p.U = pl.U;
     p.Q = split ? 1 : pl.C;
-    p.partials = split ? static_cast<float2*>(workspace) : nullptr;
-    p.counters = split ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes) : nullptr;
+    p.partials = split ? static_cast<uint2*>(workspace) : nullptr;
     // Programmatic dependent launch: the kernel may start (and prefetch its
     // weights) while the previous kernel in the stream is finishing.
     cudaLaunchConfig_t cfg = {};
@@ -709,12 +766,11 @@ extern "C" int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, cons
     void* ws = nullptr;
     rc = static_workspace_address(&ws);
     if (rc != SKINNY_OK) return rc;
-    // The array keeps whatever the previous call left; the arrival counters of
-    // this call must start at zero, so clear them on the call's stream.
-    const size_t counter_bytes = pl.workspace_bytes - pl.partial_bytes;
+    // A completed call leaves every partial-sum slot zero, but one whose
+    // device-side wait gave up may not: clear the slots this call uses, on
+    // the call's stream, so every call starts from the same state.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + pl.partial_bytes, 0, counter_bytes, st) != cudaSuccess)
-        return SKINNY_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, pl.workspace_bytes, st) != cudaSuccess) return SKINNY_ERR_CUDA;
     return skinny_nvfp4_gemm(x, M, K, w_packed, global_scale, N, y, out_dtype, ws, kStaticWorkspaceBytes, stream);
 }
 

@@ -124,17 +124,18 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
  * ---------------------------------------------------------------------- */
 
 /* Size of the optional split-K workspace for one GEMM of this format and
- * shape on the CURRENT device (it depends on the SM count).  A workspace lets
- * the kernel split K across CTAs so that every SM streams the same number of
- * weight bytes (a short-N shape such as 5120 x 5120 has too few 128-row tiles
- * to fill 148 SMs otherwise).  It holds FP32 partial sums followed by one
- * arrival counter per 128-row tile; the counters must be ZERO before the
- * first use and every completed call leaves them zero again, so zero-fill the
- * workspace once (cudaMemset) and reuse it.  Its layout is the same for every
- * shape on a device, so a workspace sized for the largest call serves calls of
- * any shape in turn; it must not be shared by calls that can run at the same
- * time.
- * Returns SKINNY_OK and *bytes, or SKINNY_ERR_INVALID_ARG / _CUDA. */
+ * shape on the CURRENT device (it depends on the SM count only: 4 KB per SM).
+ * A workspace lets the kernel split K across CTAs so that every SM streams
+ * the same number of weight bytes (a short-N shape such as 5120 x 5120 has
+ * too few 128-row tiles to fill 148 SMs otherwise).  It holds one slot of
+ * FP32 partial sums per CTA.  It must be ZERO-filled before its first use,
+ * and every call that completes without a device error leaves it zero again,
+ * so zero-fill it once (cudaMemset) and reuse it; after a call that set
+ * skinny_device_error(), zero-fill it again.  Its layout is the same for
+ * every shape on a device, so one workspace serves calls of any shape in
+ * turn; it must not be shared by calls that can run at the same time.
+ * Returns SKINNY_OK and *bytes, or SKINNY_ERR_INVALID_ARG / _UNSUPPORTED /
+ * _CUDA. */
 int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
 
 /* NVFP4 weight-only GEMM: y = x . W^T with W from skinny_pack_nvfp4.
@@ -147,7 +148,7 @@ int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
  *   y            device [M][N], FP16 (RNE) or FP32 per out_dtype, 4-byte aligned.
  *   workspace    device or NULL; if non-NULL, at least
  *                skinny_workspace_bytes(SKINNY_FMT_NVFP4, M, N, K) bytes,
- *                16-byte aligned, counters zero (see above).  NULL selects
+ *                16-byte aligned, zero-filled (see above).  NULL selects
  *                whole-tile scheduling (no split-K, nothing written besides y).
  *   stream       cudaStream_t.
  * Rounding: products of decoded weights and x are exact; only the FP32
@@ -179,13 +180,15 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
  * scratch lives in one static device array of skinny_static_workspace_capacity()
  * bytes (4 MiB) that every GPU which loads this library holds until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
- * allocating library routine.  Shapes whose scratch would not fit (more than
- * about 745k 128-row tiles on a 148-SM B200) return SKINNY_ERR_UNSUPPORTED.
+ * allocating library routine.  The scratch needed is 4 KB per SM, whatever
+ * the shape; a device with more SMs than the array has slots for returns
+ * SKINNY_ERR_UNSUPPORTED.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, which may load the library's device code); make that
  * first call outside any stream capture.  Every call enqueues, on `stream`, a
- * clear of the arrival counters it uses, then the GEMM.  All calls on a device
+ * clear of the partial-sum slots it uses (so a call that follows one with a
+ * device error starts clean), then the GEMM.  All calls on a device
  * share the one array, so calls that can overlap on the GPU (different
  * streams, or concurrent graph branches) race and corrupt each other's
  * results: serialise them. */
@@ -197,8 +200,10 @@ size_t skinny_static_workspace_capacity(void);
 
 /* Device-side error word of the current device.  Every wait inside the
  * kernels is bounded; a wait that gives up sets a bit here instead of
- * hanging (1 = consumer wait, 2 = producer wait, 4 = drain wait) and its CTA
- * returns early, leaving y incomplete.  Synchronises the device, stores the
+ * hanging (1 = wait for a weight tile, 2 = wait for a free ring slot,
+ * 4 = drain of copies in flight after an abort, 8 = split-K finisher waiting
+ * for another CTA's partial sums) and its CTA winds down, leaving y
+ * incomplete.  Synchronises the device, stores the
  * word in *flags and, if clear != 0, resets it.  Returns SKINNY_OK or
  * SKINNY_ERR_CUDA. */
 int skinny_device_error(int clear, unsigned* flags);

@@ -45,7 +45,7 @@ def sample_rows(N, count, seed=0):
         return np.arange(N)
     rng = np.random.default_rng(seed)
     fixed = np.concatenate([np.arange(min(16, N)), np.arange(max(0, N - 16), N),
-                            np.arange(255, N, 256)[:64], np.arange(256, N, 256)[:64]])
+                            np.arange(127, N, 128)[:64], np.arange(128, N, 128)[:64]])
     rest = rng.choice(N, size=max(0, count - fixed.size), replace=False)
     return np.unique(np.concatenate([fixed, rest]))
 

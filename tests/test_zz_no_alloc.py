@@ -60,8 +60,9 @@ def test_static_workspace_matches_allocating_entry_point(first, second):
 def test_static_workspace_rejects_oversized_shape():
     cap = sk.library().skinny_static_workspace_capacity()
     assert cap == 4 << 20
-    # More 256-row tiles than the counters region can hold after the partials.
-    n_big = 1 << 30
-    st = sk.library().skinny_nvfp4_gemm_static_ws(1 << 20, 1, 16, 1 << 20, ctypes.c_float(1.0), n_big, 1 << 20,
+    # 2^23 row tiles x 2^21 K tiles: more tiles than the kernel's schedule can
+    # index.  The call is refused before anything touches the (fake) pointers.
+    big = 1 << 30
+    st = sk.library().skinny_nvfp4_gemm_static_ws(1 << 20, 1, big, 1 << 20, ctypes.c_float(1.0), big, 1 << 20,
                                                   sk.OUT_F32, None)
     assert st == sk.ERR_UNSUPPORTED
