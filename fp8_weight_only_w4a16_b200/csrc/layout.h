@@ -39,7 +39,7 @@ constexpr int kNvfp4TileBytes = kNvfp4TileCodeBytes + kNvfp4TileScaleBytes;
 constexpr int kFp8TileBytes = kTileRows * kTileK;                 // 65536
 constexpr int kNvfp4StripCodeBytes = kChunks * 512;   // one strip: 8 chunks x 32 lanes x 16 bytes
 constexpr int kNvfp4StripScaleBytes = kChunks * 64;   // one strip: 8 chunks x 64 scale bytes
-constexpr int kFp8StripBytes = kChunks * 1024;        // one strip: 8 chunks x 32 lanes x 32 bytes
+constexpr int kFp8StripBytes = kChunks * 1024;        // one strip: 8 chunks x 2 halves x 32 lanes x 16 bytes
 
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
@@ -88,16 +88,20 @@ inline int nvfp4_scale_offset(int r, int b)
 }
 
 // Byte offset, inside a 65536-byte FP8 tile, of element (row r, column k).
-// A lane's 32 bytes per chunk: step j in bytes 8j..8j+7, register r in bytes
-// 2r, 2r+1, element e in byte e (cvt.rn.f16x2.e4m3x2 turns the low byte into
-// the low half).
+// A lane's 32 bytes per chunk are two 16-byte halves 512 bytes apart (steps
+// j = 0, 1 in the first, j = 2, 3 in the second), so that each 16-byte
+// shared-memory load of a warp reads 512 contiguous bytes (no bank
+// conflicts).  Inside a half: step j in bytes 8(j%2)..8(j%2)+7, register r in
+// bytes 2r, 2r+1, element e in byte e (cvt.rn.f16x2.e4m3x2 turns the low byte
+// into the low half).
 inline int fp8_offset(int r, int k)
 {
     const Slot s = tile_slot(r, k);
     const int strip = r / 16, rr = r % 16;
     const int gid = rr % 8;
     const int ch = k / 64, t = (k % 64) / 16;
-    return strip * kFp8StripBytes + ch * 1024 + (4 * gid + t) * 32 + 8 * s.j + 2 * s.reg + s.e;
+    return strip * kFp8StripBytes + ch * 1024 + (s.j / 2) * 512 + (4 * gid + t) * 16 + 8 * (s.j % 2) + 2 * s.reg +
+           s.e;
 }
 
 }  // namespace skinny

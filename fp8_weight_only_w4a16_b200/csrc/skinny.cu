@@ -376,7 +376,7 @@ struct Consumer {
                 for (int q = 0; q < 2; ++q) {
                     const uint32_t base = tile + lane_codes + q * kFp8StripBytes + u * 1024;
                     cw[u][q][0] = ptx::lds128(base);
-                    cw[u][q][1] = ptx::lds128(base + 16);
+                    cw[u][q][1] = ptx::lds128(base + 512);
                 }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -411,7 +411,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         w.lane_codes = (2 * sp) * kNvfp4StripCodeBytes + (2 * kq) * 512 + lane * 16;
         w.lane_scale = Tile<FMT>::kScalesOff + (2 * sp) * kNvfp4StripScaleBytes + (2 * kq) * 64 + t * 16 + gid * 2;
     } else {
-        w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 32;
+        w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 16;
         w.lane_scale = 0;
     }
     // Activations: token gid, columns c*512 + (2kq + u)*64 + [16t, 16t+16).

@@ -128,13 +128,14 @@ def test_fp8_lane_bytes_hold_their_slots():
         for chunk in range(8):
             for lane in range(32):
                 gid, t = lane // 4, lane % 4
-                base = strip * 8192 + chunk * 1024 + lane * 32
                 for j in range(4):
+                    # two 16-byte halves per lane, 512 bytes apart (conflict-free loads)
+                    base = strip * 8192 + chunk * 1024 + (j // 2) * 512 + lane * 16 + 8 * (j % 2)
                     for r in range(4):
                         for e in range(2):
                             row = strip * 16 + gid + 8 * (r & 1)
                             col = chunk * 64 + 16 * t + 4 * j + 2 * (r >> 1) + e
-                            assert pc[base + 8 * j + 2 * r + e] == q[row, col]
+                            assert pc[base + 2 * r + e] == q[row, col]
 
 
 def test_pack_rejects_bad_scale_bytes():
