@@ -276,6 +276,70 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3):
     return out
 
 
+def lm_head_argmax_us(dev, launches: int = 20, replays: int = 3):
+    """Per-launch device time of the vocabulary projection 151936 x 5120 (NVFP4)
+    fused with the per-token argmax, next to the same GEMM writing FP32 logits,
+    at M = 1 and 8 (graphs of back-to-back launches over weight copies > 4x L2).
+    The packed bytes are drawn directly on the device: random E2M1 codes and
+    UE4M3 block scales in [2^-4, 2^4], one valid tile layout per copy."""
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+    from fp8_weight_only_w4a16_b200 import PackedNVFP4
+
+    N, K = 151936, 5120
+    nbytes = sk.nvfp4_packed_bytes(N, K)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_copy = max(2, int(np.ceil(4 * l2 / nbytes)))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    copies = []
+    for _ in range(n_copy):
+        t = torch.randint(0, 256, (nbytes // 36864, 36864), dtype=torch.uint8, device=dev, generator=gen)
+        t[:, 32768:] = torch.randint(0x18, 0x59, (nbytes // 36864, 4096), dtype=torch.uint8, device=dev,
+                                     generator=gen)
+        copies.append(PackedNVFP4(t.view(-1), 1.0, N, K))
+    ws = sk.make_workspace(sk.FMT_NVFP4, 8, N, K, dev)
+    out = []
+    stream = torch.cuda.Stream()
+    for M in PASSES:
+        x = torch.randn((M, K), generator=gen, device=dev).to(torch.float16)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        idx = torch.empty((M,), dtype=torch.int32, device=dev)
+        val = torch.empty((M,), dtype=torch.float32, device=dev)
+        row = {"M": M}
+        for kind in ("fused_argmax", "gemm_fp32"):
+            def one(w):
+                if kind == "fused_argmax":
+                    sk.gemm_argmax_into(idx, val, x, w, ws)
+                else:
+                    sk.gemm_into(y, x, w, workspace=ws)
+            stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(stream):
+                one(copies[0])
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for r in range(launches):
+                    one(copies[r % n_copy])
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(replays):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / (replays * launches)
+            alg = nbytes + 4 + M * K * 2 + (M * 8 if kind == "fused_argmax" else M * N * 4)
+            row[kind] = {"us": round(us, 3), "GB/s": round(alg / us / 1e3, 1)}
+            del g
+        out.append(row)
+    del copies, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def launch_one(y, x, w, ws):
     import fp8_weight_only_w4a16_b200 as sk
 
@@ -494,6 +558,7 @@ def main(argv=None):
     # Per-launch device time of each GEMM (CUDA events around graphs of
     # back-to-back launches); this also brings the GPU to its loaded clocks.
     dur_us = per_launch_us(weights, xs, ys, ws)
+    lm_head = lm_head_argmax_us(dev)
 
     for i in range(args.warmup):
         graphs[i % COPIES].replay()
@@ -557,6 +622,9 @@ def main(argv=None):
                                "launches"},
         "sum_launch_us": round(float(dur_us.sum()), 2),
         "per_gemm": per,
+        "lm_head_argmax": {"gemm": "lm_head nvfp4 151936x5120", "note": "fused per-token argmax (no logits "
+                           "written) vs the same GEMM writing FP32 logits; per-launch device time, not part of the "
+                           "step", "passes": lm_head},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(PASSES) * len(si.MIXED_LAYER) * args.steps,
         "clocks": clocks,

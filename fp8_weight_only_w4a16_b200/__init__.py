@@ -68,6 +68,8 @@ def library() -> ctypes.CDLL:
                 "skinny_device_error": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint)]),
                 "skinny_nvfp4_gemm_static_ws": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
                                                                ctypes.c_int, p]),
+                "skinny_nvfp4_gemm_argmax": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p, p,
+                                                            sz, p]),
                 "skinny_static_workspace_capacity": (sz, []),
             }
             for name, (res, args) in sigs.items():
@@ -250,6 +252,37 @@ def gemm(x, w, out_dtype=None, workspace=None, stream=None):
     y = torch.empty((x.shape[0], w.N), dtype=out_dtype or torch.float16, device=x.device)
     gemm_into(y, x, w, workspace=workspace, stream=stream)
     return y
+
+
+def gemm_argmax_into(idx, val, x, w, workspace, stream=None) -> None:
+    """Per token m: idx[m] = argmax_n y[m, n], val[m] = y[m, idx[m]] for y = x . W^T
+    (NVFP4 W), without writing y.  idx int32 [M], val float32 [M]; the workspace
+    (zero-filled, from make_workspace) is required."""
+    import torch
+
+    M, K = x.shape
+    if x.dtype != torch.float16 or not x.is_contiguous() or K != w.K:
+        raise ValueError("x must be a contiguous float16 [M, %d] tensor" % w.K)
+    if w.fmt != FMT_NVFP4:
+        raise ValueError("the fused argmax takes NVFP4 weights")
+    if idx.shape != (M,) or idx.dtype != torch.int32 or val.shape != (M,) or val.dtype != torch.float32:
+        raise ValueError("idx must be int32 [M] and val float32 [M]")
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = library().skinny_nvfp4_gemm_argmax(x.data_ptr(), M, K, w.data.data_ptr(), ctypes.c_float(w.global_scale),
+                                            w.N, idx.data_ptr(), val.data_ptr(), ws_ptr, ws_bytes,
+                                            _stream_handle(stream))
+    _check(st, "skinny_nvfp4_gemm_argmax")
+
+
+def gemm_argmax(x, w, workspace, stream=None):
+    """Allocate and return (idx int32 [M], val float32 [M]): see gemm_argmax_into."""
+    import torch
+
+    idx = torch.empty((x.shape[0],), dtype=torch.int32, device=x.device)
+    val = torch.empty((x.shape[0],), dtype=torch.float32, device=x.device)
+    gemm_argmax_into(idx, val, x, w, workspace, stream=stream)
+    return idx, val
 
 
 def device_error(clear: bool = True) -> int:

@@ -191,6 +191,22 @@ __device__ __forceinline__ uint2 ld_volatile_v2(const uint2* p)
     return v;
 }
 
+// Ticket of the fused-argmax completion: release this CTA's atomics (ordered
+// before it by the preceding CTA barrier) and acquire the other CTAs'.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v)
+{
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -78,6 +78,10 @@ constexpr unsigned kErrPartialWait = 8u;   // a finisher waiting for a partial s
 
 __device__ unsigned int g_device_error;
 
+// Fused argmax: this CTA's best key per token, folded into the global maxima
+// once, at the end of the kernel.
+__shared__ unsigned long long s_argmax_best[SKINNY_MAX_M];
+
 template <int FMT>
 struct Tile;
 
@@ -126,6 +130,12 @@ struct Params {
     int U;                        // tiles in total (G * C)
     int Q;                        // scheduling quantum: 1 (split K) or C (whole row tiles)
     int out_f32;
+    // Fused argmax (instead of storing y): each token's largest output and its row.
+    int argmax;
+    unsigned long long* amax_key; // [SKINNY_MAX_M] running maxima, zero between calls
+    int* amax_done;               // CTAs that have finished, zero between calls
+    int* out_idx;                 // [M]
+    float* out_val;               // [M]
 };
 
 // CTA b of P takes quanta [b*UQ/P, (b+1)*UQ/P) of the UQ = U/Q quanta.
@@ -176,15 +186,55 @@ __device__ __forceinline__ uint32_t encode_partial(float v)
 
 __device__ __forceinline__ float decode_partial(uint32_t e) { return __uint_as_float(~e); }
 
+// Argmax keys: 64 bits that order (value, row) pairs as "larger value first,
+// then smaller row".  The value's bits are mapped to an unsigned integer in
+// the order of the floats (NaN, made canonical, above +inf; -0 made +0); the
+// row is stored complemented.  Every real key is above zero, so a zero key
+// means "no candidate yet".
+__device__ __forceinline__ unsigned long long argmax_key(float v, int n)
+{
+    if (v != v) v = __uint_as_float(0x7FC00000u);
+    if (v == 0.f) v = 0.f;
+    const uint32_t b = __float_as_uint(v);
+    const uint32_t u = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (uint32_t)n);
+}
+
+__device__ __forceinline__ float argmax_key_value(unsigned long long key)
+{
+    const uint32_t u = (uint32_t)(key >> 32);
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+__device__ __forceinline__ int argmax_key_row(unsigned long long key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
+
 // One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
-// tokens 2t and 2t+1 of this lane (v[0], v[1]).
+// tokens 2t and 2t+1 of this lane (v[0], v[1]).  Called by all 32 lanes.
 template <int FMT>
 __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane)
 {
     const int gid = lane >> 2, t = lane & 3;
     const int n = g * kTileRows + strip * kStripRows + gid + 8 * h;
+    const float sc = (FMT == SKINNY_FMT_NVFP4) ? p.out_scale : (n < p.N ? p.channel_scale[n] : 0.f);
+    if (p.argmax) {
+        // The warp's best (value, row) per token: lanes with the same t hold
+        // the same two tokens for eight rows; one shared-memory atomic per
+        // token per warp, one global atomic per token per CTA (at the end).
+        // The value is the one the FP32-output GEMM would store.
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int m = 2 * t + e;
+            unsigned long long key = (n < p.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
+#pragma unroll
+            for (int d = 4; d < 32; d <<= 1) {
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, d);
+                key = o > key ? o : key;
+            }
+            if (gid == 0 && key != 0ull) atomicMax(&s_argmax_best[m], key);
+        }
+        return;
+    }
     if (n >= p.N) return;
-    const float sc = (FMT == SKINNY_FMT_NVFP4) ? p.out_scale : p.channel_scale[n];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int m = 2 * t + e;
@@ -515,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Sched sc = make_sched(p, blockIdx.x, gridDim.x);
 
+    if (threadIdx.x < SKINNY_MAX_M) s_argmax_best[threadIdx.x] = 0ull;
     if (threadIdx.x == 0) {
         ptx::pdl_launch_dependents();
         for (int s = 0; s < S::kStages; ++s) {
@@ -533,6 +584,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     ptx::pdl_wait_prior_grid();
 
     consume<FMT>(p, smem, full, empty, sc, warp, lane);
+
+    if (p.argmax) {
+        // The CTA that finishes last turns the maxima into (row, value) per
+        // token and leaves the keys and the counter at zero for the next call.
+        __shared__ int last_cta;
+        __syncthreads();   // every warp's shared-memory maxima are in
+        if (threadIdx.x < p.M && s_argmax_best[threadIdx.x] != 0ull)
+            atomicMax(&p.amax_key[threadIdx.x], s_argmax_best[threadIdx.x]);
+        __syncthreads();   // this CTA's global atomics are issued
+        if (threadIdx.x == 0)
+            last_cta = ptx::atomic_add_acq_rel_gpu(p.amax_done, 1) == (int)gridDim.x - 1;
+        __syncthreads();
+        if (last_cta && threadIdx.x < p.M) {
+            const unsigned long long key = ptx::ld_volatile_u64(&p.amax_key[threadIdx.x]);
+            p.out_idx[threadIdx.x] = argmax_key_row(key);
+            p.out_val[threadIdx.x] = argmax_key_value(key);
+            p.amax_key[threadIdx.x] = 0ull;
+        }
+        if (last_cta && threadIdx.x == 0) *p.amax_done = 0;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -573,10 +644,12 @@ static int current_device(int* sms)
 
 // Workspace layout (identical for every shape on a device, so one workspace
 // can serve calls of different shapes in turn): one partial-sum slot of
-// 16 warps x 32 lanes x 2 floats per CTA, for up to one CTA per SM.
+// 16 warps x 32 lanes x 2 floats per CTA, for up to one CTA per SM, then the
+// fused argmax's running maxima (one 64-bit key per token) and CTA counter.
+constexpr size_t kArgmaxTailBytes = 256;
 struct Plan {
     int G, C, U, P;
-    size_t workspace_bytes;
+    size_t partial_bytes, workspace_bytes;
 };
 
 static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* pl)
@@ -590,7 +663,8 @@ static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* p
     pl->U = (int)(G * C);
     const int UQ = split ? pl->U : pl->G;
     pl->P = UQ < sms ? UQ : sms;
-    pl->workspace_bytes = (size_t)sms * kConsumerWarps * 32 * sizeof(uint2);
+    pl->partial_bytes = (size_t)sms * kConsumerWarps * 32 * sizeof(uint2);
+    pl->workspace_bytes = pl->partial_bytes + kArgmaxTailBytes;
     return SKINNY_OK;
 }
 
@@ -623,6 +697,12 @@ static int launch(Params p, int64_t N, int64_t K, void* workspace, size_t worksp
     p.U = pl.U;
     p.Q = split ? 1 : pl.C;
     p.partials = split ? static_cast<uint2*>(workspace) : nullptr;
+    if (p.argmax) {
+        if (!split) return SKINNY_ERR_WORKSPACE;
+        uint8_t* tail = static_cast<uint8_t*>(workspace) + pl.partial_bytes;
+        p.amax_key = reinterpret_cast<unsigned long long*>(tail);
+        p.amax_done = reinterpret_cast<int*>(tail + SKINNY_MAX_M * sizeof(unsigned long long));
+    }
     // Programmatic dependent launch: the kernel may start (and prefetch its
     // weights) while the previous kernel in the stream is finishing.
     cudaLaunchConfig_t cfg = {};
@@ -712,6 +792,29 @@ extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_pa
     p.N = (int)N;
     p.out_f32 = out_dtype == SKINNY_OUT_F32;
     return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
+                                        int64_t N, int32_t* argmax_idx, float* argmax_val, void* workspace,
+                                        size_t workspace_bytes, void* stream)
+{
+    int rc = check_common(x, M, K, N, argmax_val, SKINNY_OUT_F32, workspace);
+    if (rc != SKINNY_OK) return rc;
+    if (!w_packed || !argmax_idx) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(w_packed, 16) || !aligned(argmax_idx, 4)) return SKINNY_ERR_ALIGNMENT;
+    if (!workspace) return SKINNY_ERR_WORKSPACE;
+    Params p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = static_cast<const uint8_t*>(w_packed);
+    p.out_scale = global_scale;
+    p.M = M;
+    p.K = (int)K;
+    p.N = (int)N;
+    p.out_f32 = 1;
+    p.argmax = 1;
+    p.out_idx = argmax_idx;
+    p.out_val = argmax_val;
+    return launch<SKINNY_FMT_NVFP4>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

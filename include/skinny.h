@@ -124,7 +124,8 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
  * ---------------------------------------------------------------------- */
 
 /* Size of the optional split-K workspace for one GEMM of this format and
- * shape on the CURRENT device (it depends on the SM count only: 4 KB per SM).
+ * shape on the CURRENT device (it depends on the SM count only: 4 KB per SM
+ * plus 256 bytes for the fused argmax's running maxima).
  * A workspace lets the kernel split K across CTAs so that every SM streams
  * the same number of weight bytes (a short-N shape such as 5120 x 5120 has
  * too few 128-row tiles to fill 148 SMs otherwise).  It holds one slot of
@@ -165,6 +166,27 @@ int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_packed, flo
 int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
                     const float* channel_scale, int64_t N, void* y, int out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* NVFP4 GEMM fused with a per-token argmax over the N outputs: the greedy
+ * pick of an lm_head (vocabulary projection), or the local argmax of a
+ * speculative-verify round, without writing the M x N logits.  (Taozi.news
+ * article, section "自研 QPN 内核", and the aiwitness.kr post, section
+ * "내가 실제로 만든 것": the drafter and the verify round take the greedy /
+ * local argmax of the vocabulary projection.)
+ *   argmax_idx   device int32[M]: for token m, the row n with the largest
+ *                y[m][n]; ties go to the smallest n, a NaN output counts as
+ *                larger than any number (as torch.argmax), -0.0 equals +0.0.
+ *   argmax_val   device float[M]: that y[m][n], bitwise the value the FP32
+ *                output of skinny_nvfp4_gemm would hold with the same
+ *                workspace size (same schedule and summation order).
+ *   workspace    REQUIRED (the running maxima live in its tail); sized and
+ *                zero-filled as for skinny_nvfp4_gemm, and left zero again.
+ * Other arguments as skinny_nvfp4_gemm.  A NULL workspace returns
+ * SKINNY_ERR_WORKSPACE; null or unaligned outputs return INVALID_ARG /
+ * ALIGNMENT.  The outputs are written by one CTA at the end of the kernel. */
+int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_packed, float global_scale, int64_t N,
+                             int32_t* argmax_idx, float* argmax_val, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /* NVFP4 GEMM for callers that cannot allocate device memory.
  *

@@ -80,3 +80,21 @@ def test_workspace_query_argument_checks():
     assert lib.skinny_workspace_bytes(0, 1, 64, 40, ctypes.byref(b)) == sk.ERR_INVALID_ARG
     assert lib.skinny_workspace_bytes(0, 9, 64, 64, ctypes.byref(b)) == sk.ERR_UNSUPPORTED
     assert lib.skinny_workspace_bytes(0, 1, 64, 64, None) == sk.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(idx=None), sk.ERR_INVALID_ARG),
+    (dict(val=None), sk.ERR_INVALID_ARG),
+    (dict(w=None), sk.ERR_INVALID_ARG),
+    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(K=40), sk.ERR_INVALID_ARG),
+    (dict(idx=ALIGNED + 2), sk.ERR_ALIGNMENT),
+    (dict(val=ALIGNED + 2), sk.ERR_ALIGNMENT),
+    (dict(ws=None), sk.ERR_WORKSPACE),
+])
+def test_nvfp4_argmax_argument_checks(kw, status):
+    a = dict(x=ALIGNED, M=1, K=64, w=ALIGNED, N=32, idx=ALIGNED, val=ALIGNED, ws=ALIGNED)
+    a.update(kw)
+    st = sk.library().skinny_nvfp4_gemm_argmax(a["x"], a["M"], a["K"], a["w"], 1.0, a["N"], a["idx"], a["val"],
+                                               a["ws"], 1 << 20, None)
+    assert st == status
