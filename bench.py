@@ -276,68 +276,95 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3):
     return out
 
 
-def lm_head_argmax_us(dev, launches: int = 20, replays: int = 3):
-    """Per-launch device time of the vocabulary projection 151936 x 5120 (NVFP4)
-    fused with the per-token argmax, next to the same GEMM writing FP32 logits,
-    at M = 1 and 8 (graphs of back-to-back launches over weight copies > 4x L2).
-    The packed bytes are drawn directly on the device: random E2M1 codes and
-    UE4M3 block scales in [2^-4, 2^4], one valid tile layout per copy."""
+def _random_packed_copies(dev, N, K, gen):
+    """Packed NVFP4 tiles drawn on the device (random E2M1 codes, UE4M3 block
+    scales in [2^-4, 2^4]), as many copies as it takes to exceed 4x L2."""
     import torch
 
     import fp8_weight_only_w4a16_b200 as sk
-    from fp8_weight_only_w4a16_b200 import PackedNVFP4
 
-    N, K = 151936, 5120
     nbytes = sk.nvfp4_packed_bytes(N, K)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_copy = max(2, int(np.ceil(4 * l2 / nbytes)))
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(5)
     copies = []
     for _ in range(n_copy):
         t = torch.randint(0, 256, (nbytes // 36864, 36864), dtype=torch.uint8, device=dev, generator=gen)
         t[:, 32768:] = torch.randint(0x18, 0x59, (nbytes // 36864, 4096), dtype=torch.uint8, device=dev,
                                      generator=gen)
-        copies.append(PackedNVFP4(t.view(-1), 1.0, N, K))
-    ws = sk.make_workspace(sk.FMT_NVFP4, 8, N, K, dev)
-    out = []
+        copies.append(t.view(-1))
+    return copies, nbytes
+
+
+def _graph_us(one, n_copy, launches, replays):
+    """Average device time of one launch: a CUDA graph of back-to-back launches
+    rotating over the weight copies, CUDA events around the replays."""
+    import torch
+
     stream = torch.cuda.Stream()
-    for M in PASSES:
-        x = torch.randn((M, K), generator=gen, device=dev).to(torch.float16)
-        y = torch.empty((M, N), dtype=torch.float32, device=dev)
-        idx = torch.empty((M,), dtype=torch.int32, device=dev)
-        val = torch.empty((M,), dtype=torch.float32, device=dev)
-        row = {"M": M}
-        for kind in ("fused_argmax", "gemm_fp32"):
-            def one(w):
-                if kind == "fused_argmax":
-                    sk.gemm_argmax_into(idx, val, x, w, ws)
-                else:
-                    sk.gemm_into(y, x, w, workspace=ws)
-            stream.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(stream):
-                one(copies[0])
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for r in range(launches):
-                    one(copies[r % n_copy])
-            g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(replays):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            us = 1e3 * e0.elapsed_time(e1) / (replays * launches)
-            alg = nbytes + 4 + M * K * 2 + (M * 8 if kind == "fused_argmax" else M * N * 4)
-            row[kind] = {"us": round(us, 3), "GB/s": round(alg / us / 1e3, 1)}
-            del g
-        out.append(row)
-    del copies, ws
-    torch.cuda.empty_cache()
-    return out
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        one(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(launches):
+            one(r % n_copy)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return 1e3 * e0.elapsed_time(e1) / (replays * launches)
+
+
+def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
+    """Per-launch device time of the two fused epilogues next to the plain GEMM
+    they replace, at M = 1 and 8:
+      * the vocabulary projection 151936 x 5120 fused with the per-token argmax
+        vs the same GEMM writing FP32 logits;
+      * the gate+up projection 34816 x 5120 fused with SiLU*mul (17408 FP16
+        outputs) vs the same GEMM writing its 34816 FP16 outputs."""
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+    from fp8_weight_only_w4a16_b200 import PackedGateUp, PackedNVFP4
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    result = {}
+    for name, N, K in (("lm_head_argmax", 151936, 5120), ("gate_up_silu_mul", 34816, 5120)):
+        copies, nbytes = _random_packed_copies(dev, N, K, gen)
+        plain = [PackedNVFP4(c, 1.0, N, K) for c in copies]
+        gu = [PackedGateUp(c, 1.0 / 448, N // 2, K) for c in copies]
+        ws = sk.make_workspace(sk.FMT_NVFP4, 8, N, K, dev)
+        rows = []
+        for M in PASSES:
+            x = torch.randn((M, K), generator=gen, device=dev).to(torch.float16)
+            row = {"M": M}
+            if name == "lm_head_argmax":
+                y = torch.empty((M, N), dtype=torch.float32, device=dev)
+                idx = torch.empty((M,), dtype=torch.int32, device=dev)
+                val = torch.empty((M,), dtype=torch.float32, device=dev)
+                kinds = {"fused_argmax": (lambda c: sk.gemm_argmax_into(idx, val, x, plain[c], ws), M * 8),
+                         "gemm_fp32": (lambda c: sk.gemm_into(y, x, plain[c], workspace=ws), M * N * 4)}
+            else:
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                h = torch.empty((M, N // 2), dtype=torch.float16, device=dev)
+                kinds = {"fused_silu_mul": (lambda c: sk.gemm_silu_mul_into(h, x, gu[c], workspace=ws), M * N),
+                         "gemm_fp16": (lambda c: sk.gemm_into(y, x, plain[c], workspace=ws), M * N * 2)}
+            for kind, (one, out_bytes) in kinds.items():
+                us = _graph_us(one, len(copies), launches, replays)
+                alg = nbytes + 4 + M * K * 2 + out_bytes
+                row[kind] = {"us": round(us, 3), "GB/s": round(alg / us / 1e3, 1)}
+            rows.append(row)
+        result[name] = {"gemm": "nvfp4 %dx%d" % (N, K), "passes": rows}
+        del copies, plain, gu, ws
+        torch.cuda.empty_cache()
+    return result
 
 
 def launch_one(y, x, w, ws):
@@ -558,7 +585,7 @@ def main(argv=None):
     # Per-launch device time of each GEMM (CUDA events around graphs of
     # back-to-back launches); this also brings the GPU to its loaded clocks.
     dur_us = per_launch_us(weights, xs, ys, ws)
-    lm_head = lm_head_argmax_us(dev)
+    fused = fused_epilogues_us(dev)
 
     for i in range(args.warmup):
         graphs[i % COPIES].replay()
@@ -622,9 +649,9 @@ def main(argv=None):
                                "launches"},
         "sum_launch_us": round(float(dur_us.sum()), 2),
         "per_gemm": per,
-        "lm_head_argmax": {"gemm": "lm_head nvfp4 151936x5120", "note": "fused per-token argmax (no logits "
-                           "written) vs the same GEMM writing FP32 logits; per-launch device time, not part of the "
-                           "step", "passes": lm_head},
+        "fused_epilogues": dict(fused, note="next rows: the per-token argmax and the SiLU*mul activation fused "
+                                            "into the GEMM epilogue, each next to the plain GEMM it replaces; "
+                                            "per-launch device time, not part of the step"),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(PASSES) * len(si.MIXED_LAYER) * args.steps,
         "clocks": clocks,

@@ -70,6 +70,9 @@ def library() -> ctypes.CDLL:
                                                                ctypes.c_int, p]),
                 "skinny_nvfp4_gemm_argmax": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p, p,
                                                             sz, p]),
+                "skinny_pack_nvfp4_gate_up": (ctypes.c_int, [p, p, i64, i64, p]),
+                "skinny_nvfp4_gemm_silu_mul": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
+                                                              ctypes.c_int, p, sz, p]),
                 "skinny_static_workspace_capacity": (sz, []),
             }
             for name, (res, args) in sigs.items():
@@ -251,6 +254,62 @@ def gemm(x, w, out_dtype=None, workspace=None, stream=None):
 
     y = torch.empty((x.shape[0], w.N), dtype=out_dtype or torch.float16, device=x.device)
     gemm_into(y, x, w, workspace=workspace, stream=stream)
+    return y
+
+
+def pack_nvfp4_gate_up(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Pack gate+up weights (rows 0..F-1 gate, F..2F-1 up) for the fused SiLU*mul GEMM."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    n2, half_k = codes.shape
+    K = 2 * half_k
+    if n2 % 2 or scales.shape != (n2, K // 16):
+        raise ValueError("codes [2F, K/2] and scales [2F, K/16] expected")
+    out = np.zeros(nvfp4_packed_bytes(n2, K), np.uint8)
+    _check(library().skinny_pack_nvfp4_gate_up(codes.ctypes.data, scales.ctypes.data, n2 // 2, K, out.ctypes.data),
+           "skinny_pack_nvfp4_gate_up")
+    return out
+
+
+@dataclasses.dataclass
+class PackedGateUp:
+    """Gate+up NVFP4 weights packed for gemm_silu_mul: F outputs, 2F weight rows."""
+    data: "object"
+    global_scale: float
+    F: int
+    K: int
+
+    @classmethod
+    def from_logical(cls, codes: np.ndarray, scales: np.ndarray, global_scale: float, device="cuda"):
+        import torch
+
+        return cls(torch.from_numpy(pack_nvfp4_gate_up(codes, scales)).to(device), float(global_scale),
+                   codes.shape[0] // 2, codes.shape[1] * 2)
+
+
+def gemm_silu_mul_into(y, x, w: "PackedGateUp", workspace=None, stream=None) -> None:
+    """y[M, F] = silu(x . Wgate^T) * (x . Wup^T) (y float16 or float32, preallocated)."""
+    import torch
+
+    M, K = x.shape
+    if x.dtype != torch.float16 or not x.is_contiguous() or K != w.K:
+        raise ValueError("x must be a contiguous float16 [M, %d] tensor" % w.K)
+    if y.shape != (M, w.F) or not y.is_contiguous() or y.dtype not in (torch.float16, torch.float32):
+        raise ValueError("y must be a contiguous float16/float32 [M, F] tensor")
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_F16
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = library().skinny_nvfp4_gemm_silu_mul(x.data_ptr(), M, K, w.data.data_ptr(), ctypes.c_float(w.global_scale),
+                                              w.F, y.data_ptr(), out, ws_ptr, ws_bytes, _stream_handle(stream))
+    _check(st, "skinny_nvfp4_gemm_silu_mul")
+
+
+def gemm_silu_mul(x, w: "PackedGateUp", out_dtype=None, workspace=None, stream=None):
+    """Allocate y [M, F] and compute the fused gate+up GEMM with SiLU*mul."""
+    import torch
+
+    y = torch.empty((x.shape[0], w.F), dtype=out_dtype or torch.float16, device=x.device)
+    gemm_silu_mul_into(y, x, w, workspace=workspace, stream=stream)
     return y
 
 

@@ -104,7 +104,8 @@ struct Tile<SKINNY_FMT_FP8> {
 
 // Shared memory: kStages ring stages (one tile each), then the flush exchange
 // buffer (two parities of 16 warps x 2 strips x 32 lanes x float4), then the
-// mbarriers and the per-slot release counters.
+// mbarriers and the per-slot release counters, then (NVFP4) the buffer of the
+// fused SiLU*mul epilogue.
 template <int FMT>
 struct Smem {
     static constexpr int kStages = Tile<FMT>::kStages;
@@ -113,7 +114,10 @@ struct Smem {
     static constexpr int kXchgBytes = 2 * kConsumerWarps * 2 * 32 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
     static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
-    static constexpr int kBytes = kCountOff + kStages * 4;
+    // Fused SiLU*mul epilogue (NVFP4 only): a finished row tile's outputs, [128 rows][8 tokens] FP32.
+    static constexpr int kActOff = (kCountOff + kStages * 4 + 15) / 16 * 16;
+    static constexpr int kActBytes = FMT == SKINNY_FMT_NVFP4 ? kTileRows * SKINNY_MAX_M * 4 : 0;
+    static constexpr int kBytes = kActOff + kActBytes;
     static_assert(kStageBytes % 16 == 0, "stage alignment");
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
@@ -130,6 +134,9 @@ struct Params {
     int U;                        // tiles in total (G * C)
     int Q;                        // scheduling quantum: 1 (split K) or C (whole row tiles)
     int out_f32;
+    // Fused SiLU*mul (instead of storing y): W packed by skinny_pack_nvfp4_gate_up,
+    // y is [M][N/2] with y[m][j] = silu(gate[m][j]) * up[m][j].
+    int silu_mul;
     // Fused argmax (instead of storing y): each token's largest output and its row.
     int argmax;
     unsigned long long* amax_key; // [SKINNY_MAX_M] running maxima, zero between calls
@@ -248,6 +255,47 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
     }
 }
 
+// Fused SiLU*mul epilogue of row tile g (all 16 warps of the CTA): rows
+// 0..63 of the tile are gate rows 64g.., rows 64..127 the matching up rows,
+// so the tile yields outputs j = 64g + 0..63 of every token:
+// y[m][j] = silu(gate) * up, silu(z) = z / (1 + e^-z), in FP32.
+template <int FMT>
+__device__ void silu_mul_epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
+                                  uint8_t* smem)
+{
+    float* act = reinterpret_cast<float*>(smem + Smem<FMT>::kActOff);   // [128 rows][8 tokens]
+    const int gid = lane >> 2, t = lane & 3;
+    const int r = strip * kStripRows + gid + 8 * h;
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
+    act[r * SKINNY_MAX_M + 2 * t] = v[0] * p.out_scale;
+    act[r * SKINNY_MAX_M + 2 * t + 1] = v[1] * p.out_scale;
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
+    const int jl = threadIdx.x % 64, m = threadIdx.x / 64;          // 64 outputs x 8 tokens
+    const int F = p.N / 2, j = g * 64 + jl;
+    if (m < p.M && j < F) {
+        const float gate = act[jl * SKINNY_MAX_M + m], up = act[(64 + jl) * SKINNY_MAX_M + m];
+        const float val = gate / (1.f + expf(-gate)) * up;
+        const size_t idx = (size_t)m * F + j;
+        if (p.out_f32)
+            static_cast<float*>(p.y)[idx] = val;
+        else
+            static_cast<__half*>(p.y)[idx] = __float2half_rn(val);
+    }
+}
+
+// The finished outputs of row tile g (this warp's slice) go to y, to the
+// fused argmax, or through the fused SiLU*mul.  Called by every warp of the
+// CTA together.
+template <int FMT>
+__device__ __forceinline__ void finish(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
+                                       uint8_t* smem)
+{
+    if (FMT == SKINNY_FMT_NVFP4 && p.silu_mul)
+        silu_mul_epilogue<FMT>(p, v, g, strip, h, lane, smem);
+    else
+        epilogue<FMT>(p, v, g, strip, h, lane);
+}
+
 // Finish (or contribute to) row tile g, whose K range CTAs c_first..c_last
 // share.  The four warps of a strip pair (sp, sp+4, sp+8, sp+12) hold the
 // four K quarters of strips 2sp and 2sp+1; through shared memory each of them
@@ -277,7 +325,7 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_fi
     }
     const int strip = 2 * sp + sq;
     if (c_first == c_last) {
-        epilogue<FMT>(p, tot, g, strip, h, lane);
+        finish<FMT>(p, tot, g, strip, h, lane, smem);
         return;
     }
     if (b != c_last) {
@@ -324,7 +372,7 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_fi
     }
     sum[0] += tot[0];
     sum[1] += tot[1];
-    epilogue<FMT>(p, sum, g, strip, h, lane);
+    finish<FMT>(p, sum, g, strip, h, lane, smem);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.
@@ -792,6 +840,28 @@ extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_pa
     p.N = (int)N;
     p.out_f32 = out_dtype == SKINNY_OUT_F32;
     return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int skinny_nvfp4_gemm_silu_mul(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
+                                          int64_t F, void* y, int out_dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream)
+{
+    if (F <= 0 || F % 64 != 0) return SKINNY_ERR_INVALID_ARG;
+    int rc = check_common(x, M, K, 2 * F, y, out_dtype, workspace);
+    if (rc != SKINNY_OK) return rc;
+    if (!w_packed) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
+    Params p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = static_cast<const uint8_t*>(w_packed);
+    p.y = y;
+    p.out_scale = global_scale;
+    p.M = M;
+    p.K = (int)K;
+    p.N = (int)(2 * F);
+    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    p.silu_mul = 1;
+    return launch<SKINNY_FMT_NVFP4>(p, 2 * F, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_packed, float global_scale,

@@ -167,6 +167,29 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
                     const float* channel_scale, int64_t N, void* y, int out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Gate+up weights for the fused SiLU*mul GEMM: logical codes [2F][K/2] and
+ * scales [2F][K/16] (rows 0..F-1 = gate, F..2F-1 = up, encodings as in
+ * skinny_pack_nvfp4) are packed so that every 128-row tile holds 64 gate rows
+ * and the 64 up rows of the same outputs.  F must be a multiple of 64.
+ * w_packed: host, skinny_nvfp4_packed_bytes(2F, K) bytes.  Pure CPU.
+ * Errors: INVALID_ARG (null pointer, F % 64 != 0, bad shape, bad scale byte). */
+int skinny_pack_nvfp4_gate_up(const uint8_t* codes, const uint8_t* scales, int64_t F, int64_t K, void* w_packed);
+
+/* NVFP4 gate+up GEMM fused with the SiLU*mul activation of a gated MLP
+ * (the 34816-wide gate+up projection of the pages' model feeding its
+ * 17408-wide down projection):
+ *   y[m][j] = silu(g[m][j]) * u[m][j],  silu(z) = z / (1 + e^-z),
+ * where g = x . Wgate^T and u = x . Wup^T are the two halves of the GEMM
+ * (FP32 sums, times global_scale), evaluated in FP32 with expf and rounded
+ * once to the output type.  No M x 2F intermediate is written.
+ *   w_packed  from skinny_pack_nvfp4_gate_up (F output columns, 2F weight rows).
+ *   F         outputs per token, a multiple of 64.
+ *   y         device [M][F], FP16 or FP32 per out_dtype, 4-byte aligned.
+ *   workspace optional, sized with skinny_workspace_bytes(SKINNY_FMT_NVFP4, M, 2F, K).
+ * Other arguments and errors as skinny_nvfp4_gemm; F % 64 != 0 is INVALID_ARG. */
+int skinny_nvfp4_gemm_silu_mul(const void* x, int M, int64_t K, const void* w_packed, float global_scale, int64_t F,
+                               void* y, int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* NVFP4 GEMM fused with a per-token argmax over the N outputs: the greedy
  * pick of an lm_head (vocabulary projection), or the local argmax of a
  * speculative-verify round, without writing the M x N logits.  (Taozi.news

@@ -157,3 +157,18 @@ def nvfp4_gemm(x, codes, scales, global_scale, threads: int | None = None):
 
 def fp8_gemm(x, q, channel_scale, threads: int | None = None):
     return load().fp8_gemm(x, q, channel_scale, threads)
+
+
+def silu_mul(y_gate_up: np.ndarray) -> np.ndarray:
+    """The gated-MLP activation applied to a gate+up GEMM output, in float64.
+
+    y_gate_up is [M][2F]: columns 0..F-1 are the gate pre-activations g, columns
+    F..2F-1 the up projections u of the same outputs.  Returns [M][F] with
+    silu(g) * u, where silu(z) = z * sigmoid(z) = z / (1 + e^-z) (the SiLU of
+    the gated MLP that the gate+up projection feeds).  e^-z overflows to inf
+    for very negative z, which gives the limit silu(z) -> -0."""
+    y = np.asarray(y_gate_up, dtype=np.float64)
+    F = y.shape[1] // 2
+    g, u = y[:, :F], y[:, F:]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u

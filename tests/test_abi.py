@@ -98,3 +98,20 @@ def test_nvfp4_argmax_argument_checks(kw, status):
     st = sk.library().skinny_nvfp4_gemm_argmax(a["x"], a["M"], a["K"], a["w"], 1.0, a["N"], a["idx"], a["val"],
                                                a["ws"], 1 << 20, None)
     assert st == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(F=96), sk.ERR_INVALID_ARG),
+    (dict(F=0), sk.ERR_INVALID_ARG),
+    (dict(y=None), sk.ERR_INVALID_ARG),
+    (dict(w=None), sk.ERR_INVALID_ARG),
+    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(out=5), sk.ERR_INVALID_ARG),
+    (dict(w=ALIGNED + 4), sk.ERR_ALIGNMENT),
+])
+def test_nvfp4_silu_mul_argument_checks(kw, status):
+    a = dict(x=ALIGNED, M=2, K=64, w=ALIGNED, F=64, y=ALIGNED, out=0)
+    a.update(kw)
+    st = sk.library().skinny_nvfp4_gemm_silu_mul(a["x"], a["M"], a["K"], a["w"], 1.0, a["F"], a["y"], a["out"],
+                                                 None, 0, None)
+    assert st == status

@@ -15,6 +15,8 @@ import torch
 
 from conftest import read_golden
 
+import oracle
+
 ml_dtypes = pytest.importorskip("ml_dtypes")
 
 
@@ -290,3 +292,49 @@ def test_bad_arguments_raise(orc):
     x = np.zeros((1, 24), np.float16)
     with pytest.raises(ValueError):
         orc.nvfp4_gemm(x, np.zeros((1, 12), np.uint8), np.zeros((1, 1), np.uint8), 1.0)
+
+
+# ---------------------------------------------------------------------------
+# silu_mul: the gated-MLP activation on a gate+up output (fused SiLU*mul row)
+# ---------------------------------------------------------------------------
+
+def test_silu_mul_closed_forms():
+    """sigmoid(ln 3) = 3/4 exactly, so silu(ln 3) * u = 0.75 ln 3 * u; silu(0) = 0;
+    silu(z) -> z for large z and -> -0 for very negative z (no overflow NaN)."""
+    import math
+
+    z = np.array([[math.log(3.0), 0.0, 60.0, -800.0, 2.0, 2.0, 2.0, -3.0]])
+    h = oracle.silu_mul(z)
+    assert abs(h[0, 0] - 0.75 * math.log(3.0) * 2.0) < 1e-15
+    assert h[0, 1] == 0.0
+    assert abs(h[0, 2] - 60.0 * 2.0) < 1e-12
+    assert h[0, 3] == 0.0 and not np.isnan(h[0, 3])
+
+
+def test_silu_mul_identities():
+    """silu(z) - silu(-z) = z (sigmoid(z) + sigmoid(-z) = 1); linear in u;
+    gate and up are not interchangeable (a swapped operand fails)."""
+    rng = np.random.default_rng(3)
+    g = rng.normal(0, 4, size=(4, 64))
+    one = np.ones_like(g)
+    a = oracle.silu_mul(np.concatenate([g, one], axis=1))
+    b = oracle.silu_mul(np.concatenate([-g, one], axis=1))
+    assert np.allclose(a - b, g, rtol=0, atol=1e-12)
+    u = rng.normal(0, 1, size=g.shape)
+    h1 = oracle.silu_mul(np.concatenate([g, u], axis=1))
+    h3 = oracle.silu_mul(np.concatenate([g, 3 * u], axis=1))
+    assert np.allclose(h3, 3 * h1, rtol=1e-15, atol=0)
+    swapped = oracle.silu_mul(np.concatenate([u, g], axis=1))
+    assert not np.allclose(swapped, h1)
+
+
+def test_silu_mul_matches_torch_silu():
+    """A second implementation: torch.nn.functional.silu in float64."""
+    import torch
+
+    rng = np.random.default_rng(4)
+    g = rng.normal(0, 6, size=(3, 128))
+    u = rng.normal(0, 1, size=(3, 128))
+    want = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    got = oracle.silu_mul(np.concatenate([g, u], axis=1))
+    assert np.allclose(got, want, rtol=1e-14, atol=1e-300)

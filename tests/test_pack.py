@@ -160,3 +160,27 @@ def test_packed_bytes_reject_bad_shapes():
     assert sk.nvfp4_packed_bytes(4, 24) == 0
     assert sk.fp8_packed_bytes(4, 8) == 0
     assert sk.nvfp4_packed_bytes(5120, 5120) == 5120 * 5120 // 2 + 5120 * 5120 // 16
+
+
+@pytest.mark.parametrize("F,K", [(64, 512), (192, 1040)])
+def test_gate_up_packing_interleaves_blocks_of_64_rows(F, K):
+    """skinny_pack_nvfp4_gate_up equals the ordinary packing of the rows
+    reordered as [gate 0..63, up 0..63, gate 64..127, up 64..127, ...]."""
+    rng = np.random.default_rng(F + K)
+    codes = rng.integers(0, 256, size=(2 * F, K // 2), dtype=np.uint8)
+    scales = rng.integers(0, 0x7F, size=(2 * F, K // 16), dtype=np.uint8)
+    order = np.concatenate([np.r_[np.arange(64 * b, 64 * b + 64), F + np.arange(64 * b, 64 * b + 64)]
+                            for b in range(F // 64)])
+    want = sk.pack_nvfp4(codes[order], scales[order])
+    got = sk.pack_nvfp4_gate_up(codes, scales)
+    assert np.array_equal(got, want)
+
+
+def test_gate_up_packing_rejects_bad_shapes():
+    lib = sk.library()
+    buf = np.zeros(1 << 16, np.uint8)
+    c = np.zeros((128, 256), np.uint8)
+    s = np.zeros((128, 32), np.uint8)
+    assert lib.skinny_pack_nvfp4_gate_up(c.ctypes.data, s.ctypes.data, 96, 512, buf.ctypes.data) == sk.ERR_INVALID_ARG
+    assert lib.skinny_pack_nvfp4_gate_up(c.ctypes.data, s.ctypes.data, 64, 40, buf.ctypes.data) == sk.ERR_INVALID_ARG
+    assert lib.skinny_pack_nvfp4_gate_up(None, s.ctypes.data, 64, 512, buf.ctypes.data) == sk.ERR_INVALID_ARG
