@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -95,10 +96,14 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code: comments and whitespace are dropped,
+    so a comment edit keeps a traffic record taken on the same code valid."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "fp8_weight_only_w4a16_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "fp8_weight_only_w4a16_b200", "csrc", name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S)
+        h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

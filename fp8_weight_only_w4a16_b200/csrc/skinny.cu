@@ -38,6 +38,9 @@
 //    reproducible -- and zeroes the slots again.  No atomics, no fences, and
 //    each CTA publishes at most once.  Without a workspace, CTAs take whole
 //    row tiles.
+//  * Fused epilogues on the finished FP32 outputs: a per-token argmax (the
+//    greedy pick of a vocabulary projection, no logits written) and the
+//    SiLU*mul of a gated MLP (gate and up rows packed into the same tile).
 //  * Every wait is bounded (1 s of global time); a wait that gives up sets a
 //    bit in g_device_error and its CTA winds down instead of hanging.
 #include <cuda_fp16.h>
@@ -119,6 +122,7 @@ struct Smem {
     static constexpr int kActBytes = FMT == SKINNY_FMT_NVFP4 ? kTileRows * SKINNY_MAX_M * 4 : 0;
     static constexpr int kBytes = kActOff + kActBytes;
     static_assert(kStageBytes % 16 == 0, "stage alignment");
+    // 227 KB per CTA; the static shared variables (fused argmax) take 128 B more.
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
@@ -301,11 +305,14 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[2], int
 // four K quarters of strips 2sp and 2sp+1; through shared memory each of them
 // takes one quarter of the strip pair's outputs (strip 2sp + kq/2, rows
 // gid + 8*(kq%2)) and adds the four K quarters in order (a fixed order).
-//  * c_first == c_last: this CTA covered all of K; write y.
+//  * c_first == c_last: this CTA covered all of K; finish the outputs
+//    (store y, or the fused argmax / SiLU*mul).
 //  * this CTA is not c_last: publish the partial sums in this CTA's slot.
 //  * this CTA is c_last (the finisher): wait for the slots of c_first ..
-//    c_last-1, add them in CTA order and then its own sums, write y, and
-//    zero the slots for the next call.
+//    c_last-1, add them in CTA order and then its own sums, finish the
+//    outputs, and zero the slots for the next call.
+// Which case applies is the same for every warp of the CTA, so the barriers
+// of the exchange and of the fused epilogues are reached by all of them.
 template <int FMT>
 __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_first, int c_last, int parity,
                       uint8_t* smem, int b, int warp, int lane)
