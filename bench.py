@@ -491,7 +491,8 @@ def reference_arm(args):
     if rank != 0:
         return 0
     threads = oracle.default_threads()
-    per_step_s = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    # About 150 s of oracle time for the whole run, whatever K and W are.
+    per_step_s = max(0.01, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     frac = oracle_sample_frac(per_step_s, threads)
     items = _oracle_inputs(frac)
     for _ in range(args.warmup):
