@@ -354,7 +354,9 @@ def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
       * the vocabulary projection 151936 x 5120 fused with the per-token argmax
         vs the same GEMM writing FP32 logits;
       * the gate+up projection 34816 x 5120 fused with SiLU*mul (17408 FP16
-        outputs) vs the same GEMM writing its 34816 FP16 outputs."""
+        outputs) vs the same GEMM writing its 34816 FP16 outputs;
+      * the attention output projection 5120 x 5120 adding its result into
+        the FP16 residual stream in place vs the same GEMM writing y."""
     import torch
 
     import fp8_weight_only_w4a16_b200 as sk
@@ -363,7 +365,8 @@ def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
     gen = torch.Generator(device=dev)
     gen.manual_seed(5)
     result = {}
-    for name, N, K in (("lm_head_argmax", 151936, 5120), ("gate_up_silu_mul", 34816, 5120)):
+    for name, N, K in (("lm_head_argmax", 151936, 5120), ("gate_up_silu_mul", 34816, 5120),
+                       ("o_proj_residual_add", 5120, 5120)):
         copies, nbytes = _random_packed_copies(dev, N, K, gen)
         plain = [PackedNVFP4(c, 1.0, N, K) for c in copies]
         gu = [PackedGateUp(c, 1.0 / 448, N // 2, K) for c in copies]
@@ -378,10 +381,15 @@ def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
                 val = torch.empty((M,), dtype=torch.float32, device=dev)
                 kinds = {"fused_argmax": (lambda c: sk.gemm_argmax_into(idx, val, x, plain[c], ws), M * 8),
                          "gemm_fp32": (lambda c: sk.gemm_into(y, x, plain[c], workspace=ws), M * N * 4)}
-            else:
+            elif name == "gate_up_silu_mul":
                 y = torch.empty((M, N), dtype=torch.float16, device=dev)
                 h = torch.empty((M, N // 2), dtype=torch.float16, device=dev)
                 kinds = {"fused_silu_mul": (lambda c: sk.gemm_silu_mul_into(h, x, gu[c], workspace=ws), M * N),
+                         "gemm_fp16": (lambda c: sk.gemm_into(y, x, plain[c], workspace=ws), M * N * 2)}
+            else:
+                y = torch.zeros((M, N), dtype=torch.float16, device=dev)
+                kinds = {"fused_residual_add": (lambda c: sk.gemm_add_into(y, x, plain[c], y, workspace=ws),
+                                                2 * M * N * 2),
                          "gemm_fp16": (lambda c: sk.gemm_into(y, x, plain[c], workspace=ws), M * N * 2)}
             for kind, (one, out_bytes) in kinds.items():
                 us = _graph_us(one, len(copies), launches, replays)
@@ -680,9 +688,9 @@ def main(argv=None):
                                "launches"},
         "sum_launch_us": round(float(dur_us.sum()), 2),
         "per_gemm": per,
-        "fused_epilogues": dict(fused, note="next rows: the per-token argmax and the SiLU*mul activation fused "
-                                            "into the GEMM epilogue, each next to the plain GEMM it replaces; "
-                                            "per-launch device time, not part of the step"),
+        "fused_epilogues": dict(fused, note="next rows: the per-token argmax, the SiLU*mul activation and the "
+                                            "residual add fused into the GEMM epilogue, each next to the plain "
+                                            "GEMM it replaces; per-launch device time, not part of the step"),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(PASSES) * len(si.MIXED_LAYER) * args.steps,
         "clocks": clocks,

@@ -71,6 +71,10 @@ def library() -> ctypes.CDLL:
                 "skinny_nvfp4_gemm_argmax": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p, p,
                                                             sz, p]),
                 "skinny_pack_nvfp4_gate_up": (ctypes.c_int, [p, p, i64, i64, p]),
+                "skinny_nvfp4_gemm_add": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p,
+                                                         ctypes.c_int, p, sz, p]),
+                "skinny_fp8_gemm_add": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, i64, p, p, ctypes.c_int, p, sz,
+                                                       p]),
                 "skinny_nvfp4_gemm_silu_mul": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
                                                               ctypes.c_int, p, sz, p]),
                 "skinny_static_workspace_capacity": (sz, []),
@@ -246,6 +250,33 @@ def gemm_into(y, x, w, workspace=None, stream=None) -> None:
         st = lib.skinny_fp8_gemm(x.data_ptr(), M, K, w.codes.data_ptr(), w.channel_scale.data_ptr(), w.N,
                                  y.data_ptr(), out, ws_ptr, ws_bytes, h)
         _check(st, "skinny_fp8_gemm")
+
+
+def gemm_add_into(y, x, w, residual, workspace=None, stream=None) -> None:
+    """y[M, N] = x . W^T + residual, the add in FP32 before the one output
+    rounding; residual has y's shape and dtype and may be y itself."""
+    import torch
+
+    M, K = x.shape
+    if x.dtype != torch.float16 or not x.is_contiguous() or K != w.K:
+        raise ValueError("x must be a contiguous float16 [M, %d] tensor" % w.K)
+    if y.shape != (M, w.N) or not y.is_contiguous() or y.dtype not in (torch.float16, torch.float32):
+        raise ValueError("y must be a contiguous float16/float32 [M, N] tensor")
+    if residual.shape != y.shape or residual.dtype != y.dtype or not residual.is_contiguous():
+        raise ValueError("residual must be a contiguous tensor of y's shape and dtype")
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_F16
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    h = _stream_handle(stream)
+    lib = library()
+    if w.fmt == FMT_NVFP4:
+        st = lib.skinny_nvfp4_gemm_add(x.data_ptr(), M, K, w.data.data_ptr(), ctypes.c_float(w.global_scale), w.N,
+                                       residual.data_ptr(), y.data_ptr(), out, ws_ptr, ws_bytes, h)
+        _check(st, "skinny_nvfp4_gemm_add")
+    else:
+        st = lib.skinny_fp8_gemm_add(x.data_ptr(), M, K, w.codes.data_ptr(), w.channel_scale.data_ptr(), w.N,
+                                     residual.data_ptr(), y.data_ptr(), out, ws_ptr, ws_bytes, h)
+        _check(st, "skinny_fp8_gemm_add")
 
 
 def gemm(x, w, out_dtype=None, workspace=None, stream=None):

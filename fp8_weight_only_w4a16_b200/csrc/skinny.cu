@@ -131,6 +131,7 @@ struct Params {
     const uint8_t* codes;         // packed tiles (NVFP4 tiles carry their block scales)
     const float* channel_scale;   // FP8 per-output-channel scale [N]
     void* y;                      // [M][N]
+    const void* residual;         // [M][N], y's dtype, added before the output rounding (or null; may alias y)
     uint2* partials;              // [P][16 warps][32 lanes] encoded float pairs (split-K only)
     float out_scale;              // NVFP4 per-tensor scale (FP8: unused, the channel scales apply)
     int M, K, N;
@@ -250,8 +251,16 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
     for (int e = 0; e < 2; ++e) {
         const int m = 2 * t + e;
         if (m >= p.M) continue;
-        const float val = v[e] * sc;
         const size_t idx = (size_t)m * p.N + n;
+        // Rounded FP32 product, never contracted with the add below, so the
+        // fused add sees exactly the value the plain GEMM stores.
+        float val = __fmul_rn(v[e], sc);
+        // Fused residual add: one FP32 add, then the single output rounding.
+        // Each element is read and written by this thread only, so the
+        // residual may be y itself.
+        if (p.residual)
+            val = __fadd_rn(val, p.out_f32 ? static_cast<const float*>(p.residual)[idx]
+                                           : __half2float(static_cast<const __half*>(p.residual)[idx]));
         if (p.out_f32)
             static_cast<float*>(p.y)[idx] = val;
         else
@@ -841,6 +850,53 @@ extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_pa
     p.codes = static_cast<const uint8_t*>(w_packed);
     p.channel_scale = channel_scale;
     p.y = y;
+    p.out_scale = 1.0f;
+    p.M = M;
+    p.K = (int)K;
+    p.N = (int)N;
+    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int skinny_nvfp4_gemm_add(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
+                                     int64_t N, const void* residual, void* y, int out_dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream)
+{
+    if (!residual) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(residual, 4)) return SKINNY_ERR_ALIGNMENT;
+    int rc = check_common(x, M, K, N, y, out_dtype, workspace);
+    if (rc != SKINNY_OK) return rc;
+    if (!w_packed) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
+    Params p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = static_cast<const uint8_t*>(w_packed);
+    p.y = y;
+    p.residual = residual;
+    p.out_scale = global_scale;
+    p.M = M;
+    p.K = (int)K;
+    p.N = (int)N;
+    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    return launch<SKINNY_FMT_NVFP4>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int skinny_fp8_gemm_add(const void* x, int M, int64_t K, const void* w_packed, const float* channel_scale,
+                                   int64_t N, const void* residual, void* y, int out_dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream)
+{
+    if (!residual) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(residual, 4)) return SKINNY_ERR_ALIGNMENT;
+    int rc = check_common(x, M, K, N, y, out_dtype, workspace);
+    if (rc != SKINNY_OK) return rc;
+    if (!w_packed || !channel_scale) return SKINNY_ERR_INVALID_ARG;
+    if (!aligned(w_packed, 16) || !aligned(channel_scale, 4)) return SKINNY_ERR_ALIGNMENT;
+    Params p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.codes = static_cast<const uint8_t*>(w_packed);
+    p.channel_scale = channel_scale;
+    p.y = y;
+    p.residual = residual;
     p.out_scale = 1.0f;
     p.M = M;
     p.K = (int)K;

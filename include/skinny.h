@@ -167,6 +167,23 @@ int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed,
                     const float* channel_scale, int64_t N, void* y, int out_dtype,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* GEMM fused with a residual add, for the projections whose output joins
+ * the residual stream (the attention output projection and the MLP down
+ * projection of a decoder layer):
+ *   y[m][n] = (scale * sum_k w[n][k] x[m][k]) + residual[m][n]
+ * with the sum and the add in FP32 and one rounding to the output type.
+ *   residual  device [M][N] of the OUTPUT type (FP16 or FP32 per out_dtype),
+ *             4-byte aligned; it may be y itself (in-place update of the
+ *             residual stream).
+ * Other arguments and errors as skinny_nvfp4_gemm / skinny_fp8_gemm; a null
+ * residual is INVALID_ARG. */
+int skinny_nvfp4_gemm_add(const void* x, int M, int64_t K, const void* w_packed, float global_scale, int64_t N,
+                          const void* residual, void* y, int out_dtype, void* workspace, size_t workspace_bytes,
+                          void* stream);
+int skinny_fp8_gemm_add(const void* x, int M, int64_t K, const void* w_packed, const float* channel_scale, int64_t N,
+                        const void* residual, void* y, int out_dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* Gate+up weights for the fused SiLU*mul GEMM: logical codes [2F][K/2] and
  * scales [2F][K/16] (rows 0..F-1 = gate, F..2F-1 = up, encodings as in
  * skinny_pack_nvfp4) are packed so that every 128-row tile holds 64 gate rows

@@ -115,3 +115,22 @@ def test_nvfp4_silu_mul_argument_checks(kw, status):
     st = sk.library().skinny_nvfp4_gemm_silu_mul(a["x"], a["M"], a["K"], a["w"], 1.0, a["F"], a["y"], a["out"],
                                                  None, 0, None)
     assert st == status
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "fp8"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(res=None), sk.ERR_INVALID_ARG),
+    (dict(res=ALIGNED + 2), sk.ERR_ALIGNMENT),
+    (dict(y=None), sk.ERR_INVALID_ARG),
+    (dict(M=9), sk.ERR_UNSUPPORTED),
+])
+def test_gemm_add_argument_checks(fmt, kw, status):
+    a = dict(x=ALIGNED, M=2, K=64, w=ALIGNED, N=32, res=ALIGNED, y=ALIGNED)
+    a.update(kw)
+    lib = sk.library()
+    if fmt == "nvfp4":
+        st = lib.skinny_nvfp4_gemm_add(a["x"], a["M"], a["K"], a["w"], 1.0, a["N"], a["res"], a["y"], 0, None, 0, None)
+    else:
+        st = lib.skinny_fp8_gemm_add(a["x"], a["M"], a["K"], a["w"], ALIGNED, a["N"], a["res"], a["y"], 0, None, 0,
+                                     None)
+    assert st == status
