@@ -77,3 +77,53 @@ def test_planted_mistake_is_caught(tmp_path, name, old, new):
     out = oracle.compile_library(str(path), str(tmp_path / "liboracle_mutant.so"), force=True)
     failed = _battery(oracle.Oracle(out))
     assert failed, "no pin caught the planted mistake: " + name
+
+
+# ---------------------------------------------------------------------------
+# silu_mul (numpy): each plausible slip must fail one of its pins
+# ---------------------------------------------------------------------------
+
+def _silu_mutants():
+    def half(y):
+        y = np.asarray(y, dtype=np.float64)
+        F = y.shape[1] // 2
+        return y[:, :F], y[:, F:]
+
+    def exp_sign(y):            # e^+z instead of e^-z
+        g, u = half(y)
+        with np.errstate(over="ignore"):
+            return g / (1.0 + np.exp(g)) * u
+
+    def sigmoid_only(y):        # sigmoid(g) * u, the gate not multiplied back in
+        g, u = half(y)
+        with np.errstate(over="ignore"):
+            return 1.0 / (1.0 + np.exp(-g)) * u
+
+    def swapped(y):             # up and gate halves exchanged
+        g, u = half(y)
+        with np.errstate(over="ignore"):
+            return u / (1.0 + np.exp(-u)) * g
+
+    def no_mul(y):              # the up factor dropped
+        g, _ = half(y)
+        with np.errstate(over="ignore"):
+            return g / (1.0 + np.exp(-g))
+
+    def tanh_gelu(y):           # another activation in its place
+        g, u = half(y)
+        return 0.5 * g * (1.0 + np.tanh(0.7978845608 * (g + 0.044715 * g ** 3))) * u
+
+    return [("exp sign", exp_sign), ("sigmoid only", sigmoid_only), ("swapped halves", swapped),
+            ("no mul", no_mul), ("gelu", tanh_gelu)]
+
+
+@pytest.mark.parametrize("name,fn", _silu_mutants(), ids=[n for n, _ in _silu_mutants()])
+def test_silu_mul_pins_catch_mutant(name, fn, monkeypatch):
+    monkeypatch.setattr(oracle, "silu_mul", fn)
+    failed = 0
+    for pin in (pins.test_silu_mul_closed_forms, pins.test_silu_mul_identities, pins.test_silu_mul_matches_torch_silu):
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed >= 1, name
