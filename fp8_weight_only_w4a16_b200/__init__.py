@@ -317,11 +317,22 @@ class PackedGateUp:
         return cls(torch.from_numpy(pack_nvfp4_gate_up(codes, scales)).to(device), float(global_scale),
                    codes.shape[0] // 2, codes.shape[1] * 2)
 
+    @property
+    def fmt(self) -> int:
+        return FMT_NVFP4
+
+    @property
+    def N(self) -> int:
+        """Weight rows (gate and up): the GEMM's N, e.g. for workspace_bytes."""
+        return 2 * self.F
+
 
 def gemm_silu_mul_into(y, x, w: "PackedGateUp", workspace=None, stream=None) -> None:
     """y[M, F] = silu(x . Wgate^T) * (x . Wup^T) (y float16 or float32, preallocated)."""
     import torch
 
+    if not isinstance(w, PackedGateUp):
+        raise TypeError("gemm_silu_mul takes weights packed by PackedGateUp / pack_nvfp4_gate_up")
     M, K = x.shape
     if x.dtype != torch.float16 or not x.is_contiguous() or K != w.K:
         raise ValueError("x must be a contiguous float16 [M, %d] tensor" % w.K)

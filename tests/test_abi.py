@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import fp8_weight_only_w4a16_b200 as sk
@@ -134,3 +135,26 @@ def test_gemm_add_argument_checks(fmt, kw, status):
         st = lib.skinny_fp8_gemm_add(a["x"], a["M"], a["K"], a["w"], ALIGNED, a["N"], a["res"], a["y"], 0, None, 0,
                                      None)
     assert st == status
+
+
+def test_binding_rejects_bad_arguments_before_calling_the_library():
+    """The Python binding's own checks (no GPU, no library call)."""
+    import torch
+
+    w = sk.PackedNVFP4(torch.zeros(36864, dtype=torch.uint8), 1.0, 128, 512)
+    gu = sk.PackedGateUp(torch.zeros(36864, dtype=torch.uint8), 1.0, 64, 512)
+    assert gu.N == 128 and gu.fmt == sk.FMT_NVFP4
+    x32 = torch.zeros((2, 512), dtype=torch.float32)
+    x16 = torch.zeros((2, 512), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        sk.gemm_into(torch.zeros((2, 128), dtype=torch.float16), x32, w)
+    with pytest.raises(ValueError):
+        sk.gemm_into(torch.zeros((2, 64), dtype=torch.float16), x16, w)
+    with pytest.raises(TypeError):
+        sk.gemm_silu_mul_into(torch.zeros((2, 64), dtype=torch.float16), x16, w)
+    with pytest.raises(ValueError):
+        sk.gemm_argmax_into(torch.zeros(2, dtype=torch.int64), torch.zeros(2), x16, w, None)
+    with pytest.raises(ValueError):
+        sk.gemm_add_into(torch.zeros((2, 128), dtype=torch.float16), x16, w, torch.zeros((2, 128)))
+    with pytest.raises(ValueError):
+        sk.pack_nvfp4_gate_up(np.zeros((127, 256), np.uint8), np.zeros((127, 32), np.uint8))
