@@ -34,7 +34,7 @@ def _rank_main(rank, world, port, out):
 @pytest.mark.timeout(120)
 def test_max_over_ranks_and_aggregate_value_gloo():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()   # no fork of a threaded process
     mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
     assert out[0][0] == out[1][0] == 5.0
     expected = world * bench.step_bytes() * 100 / 5e-3 / 1e9
