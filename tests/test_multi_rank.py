@@ -53,3 +53,23 @@ def test_step_bytes_formula():
     assert w == 3 * (5120 * 5120 * 9 // 16 + 4) + (34816 * 5120 * 9 // 16 + 4) + (5120 * 17408 + 4 * 5120)
     act = sum(M * s.K * 2 + M * s.N * 2 for M in (1, 8) for s in bench.si.MIXED_LAYER)
     assert b == 2 * w + act
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """The DRAM traffic record is keyed by the kernel code: a comment or
+    whitespace edit keeps the key, a code edit changes it."""
+    import shutil
+
+    src = os.path.join(bench.ROOT, "fp8_weight_only_w4a16_b200", "csrc")
+    dst = tmp_path / "fp8_weight_only_w4a16_b200" / "csrc"
+    dst.mkdir(parents=True)
+    for name in bench.KERNEL_SOURCES:
+        shutil.copy(os.path.join(src, name), dst / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_source_hash()
+    layout = dst / "layout.h"
+    text = layout.read_text()
+    layout.write_text("// a new comment\n" + text.replace("\n", "\n\n", 3) + "/* trailing */\n")
+    assert bench.kernel_source_hash() == base
+    layout.write_text(text.replace("constexpr int kTileRows = 128;", "constexpr int kTileRows = 64;"))
+    assert bench.kernel_source_hash() != base
