@@ -82,7 +82,8 @@ int skinny_version(void);
  * The kernels read W in a private tiled order: tiles of 128 output rows x
  * 512 columns, consecutive in memory along K then N, so that a run of tiles is
  * one contiguous bulk copy and each lane of a warp finds its tensor-core
- * operand bytes in one 16-byte word.  An NVFP4 tile carries its UE4M3 block
+ * operand bytes in one 16-byte word (NVFP4) or two (FP8), read without
+ * shared-memory bank conflicts.  An NVFP4 tile carries its UE4M3 block
  * scales (32 KB codes + 4 KB scales); an FP8 tile is 64 KB.  Rows are padded
  * to a multiple of 128 and K to a multiple of 512 with zero codes and zero
  * scales, which contribute nothing.  The caller packs once per weight and
