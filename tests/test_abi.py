@@ -158,3 +158,19 @@ def test_binding_rejects_bad_arguments_before_calling_the_library():
         sk.gemm_add_into(torch.zeros((2, 128), dtype=torch.float16), x16, w, torch.zeros((2, 128)))
     with pytest.raises(ValueError):
         sk.pack_nvfp4_gate_up(np.zeros((127, 256), np.uint8), np.zeros((127, 32), np.uint8))
+
+
+def test_library_sources_allocate_no_device_memory():
+    """The weights are never dequantised into a full copy: the library makes
+    no device allocation at all (every buffer is the caller's, and the one
+    static array is the documented split-K scratch of the allocation-free
+    entry point)."""
+    csrc = os.path.join(ROOT, "fp8_weight_only_w4a16_b200", "csrc")
+    calls = re.compile(r"\b(cudaMalloc\w*|cudaMallocAsync|cudaMallocManaged|cudaMallocPitch|cuMemAlloc\w*|cuMemCreate|"
+                       r"cudaHostAlloc|malloc|new\s+\w+\s*\[)\s*\(?")
+    for name in sorted(os.listdir(csrc)):
+        text = open(os.path.join(csrc, name)).read()
+        code = re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S)
+        assert not calls.search(code), (name, calls.search(code).group(0))
+    skinny_cu = open(os.path.join(csrc, "skinny.cu")).read()
+    assert len(re.findall(r"static __device__ __align__\(256\) unsigned char g_static_workspace", skinny_cu)) == 1
