@@ -71,6 +71,8 @@ def library() -> ctypes.CDLL:
                 "skinny_nvfp4_gemm_argmax": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p, p,
                                                             sz, p]),
                 "skinny_pack_nvfp4_gate_up": (ctypes.c_int, [p, p, i64, i64, p]),
+                "skinny_debug_schedule": (ctypes.c_int, [i64, i64, ctypes.c_int, ctypes.c_int, p, ctypes.c_int,
+                                                         ctypes.POINTER(ctypes.c_int)]),
                 "skinny_nvfp4_gemm_add": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p, p,
                                                          ctypes.c_int, p, sz, p]),
                 "skinny_fp8_gemm_add": (ctypes.c_int, [p, ctypes.c_int, i64, p, p, i64, p, p, ctypes.c_int, p, sz,

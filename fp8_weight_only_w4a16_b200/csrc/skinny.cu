@@ -175,7 +175,7 @@ struct Sched {
     int last_owner;   // highest contributor of row tile last_g
 };
 
-__device__ __forceinline__ Sched make_sched(const Params& p, int b, int P)
+__host__ __device__ __forceinline__ Sched make_sched(const Params& p, int b, int P)
 {
     const int UQ = p.U / p.Q;
     Sched s;
@@ -816,6 +816,34 @@ extern "C" int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size
     rc = make_plan(fmt, N, K, sms, true, &pl);
     if (rc != SKINNY_OK) return rc;
     *bytes = pl.workspace_bytes;
+    return SKINNY_OK;
+}
+
+// The stream-K schedule the kernels compute, evaluated on the host for
+// tests: for each CTA b, out[6b..6b+5] = (u_last, n_units, first_g, last_g,
+// first_owner, last_owner).  *ctas receives the grid size.
+extern "C" int skinny_debug_schedule(int64_t N, int64_t K, int sms, int split, int* out, int cap, int* ctas)
+{
+    if (!out || !ctas || sms <= 0 || N <= 0 || K <= 0 || K % 16 != 0) return SKINNY_ERR_INVALID_ARG;
+    Plan pl;
+    const int rc = make_plan(SKINNY_FMT_NVFP4, N, K, sms, split != 0, &pl);
+    if (rc != SKINNY_OK) return rc;
+    *ctas = pl.P;
+    if (pl.P > cap) return SKINNY_ERR_WORKSPACE;
+    Params p{};
+    p.C = pl.C;
+    p.U = pl.U;
+    p.Q = split ? 1 : pl.C;
+    for (int b = 0; b < pl.P; ++b) {
+        const Sched sc = make_sched(p, b, pl.P);
+        int* o = out + 6 * b;
+        o[0] = sc.u_last;
+        o[1] = sc.n_units;
+        o[2] = sc.first_g;
+        o[3] = sc.last_g;
+        o[4] = sc.first_owner;
+        o[5] = sc.last_owner;
+    }
     return SKINNY_OK;
 }
 

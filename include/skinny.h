@@ -258,6 +258,15 @@ int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_pack
 int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
                                 int64_t N, void* y, int out_dtype, void* stream);
 
+/* Test hook (host only, no CUDA call): the stream-K schedule the GEMM kernels
+ * use for an N x K weight on a device with `sms` SMs, with split-K (split != 0,
+ * as with a workspace) or whole row tiles.  For each CTA b of the grid,
+ * out[6b .. 6b+5] = (last tile of its range, tiles in its range, first row
+ * tile, last row tile, lowest CTA sharing the first row tile, highest CTA
+ * sharing the last row tile); tiles are numbered row tile * ceil(K/512) + K
+ * tile.  *ctas receives the grid size; SKINNY_ERR_WORKSPACE if it exceeds cap. */
+int skinny_debug_schedule(int64_t N, int64_t K, int sms, int split, int* out, int cap, int* ctas);
+
 /* Size in bytes of the static scratch array used by skinny_nvfp4_gemm_static_ws. */
 size_t skinny_static_workspace_capacity(void);
 
