@@ -222,6 +222,18 @@ def _padded(nbytes: int) -> int:
     return (nbytes + 255) // 256 * 256
 
 
+def bench_config(world: int) -> dict:
+    """The workload description both arms print (the reference arm times the
+    same workload on a row sample, which its cpu_baseline.sample states)."""
+    return {"workload": WORKLOAD,
+            "gemms": ["%s %s %dx%d" % (s.name, s.fmt, s.N, s.K) for s in si.MIXED_LAYER],
+            "M": list(PASSES), "operands": "NVFP4/FP8 weights x FP16 activations, FP32 accumulation",
+            "l2": "inputs larger than L2: %d rotating weight copies, %.0f MB" %
+                  (COPIES, COPIES * sum(weight_bytes(s) for s in si.MIXED_LAYER) / 1e6),
+            "bytes_per_step": step_bytes(), "launch": "CUDA graph per step",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
 def copy_for(step: int, pass_idx: int) -> int:
     return (2 * step + pass_idx) % COPIES
 
@@ -261,18 +273,21 @@ def clone_weight(w):
     return sk.PackedFP8(w.codes.clone(), w.channel_scale, w.N, w.K)
 
 
-def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3):
-    """Average device time of one launch of each GEMM of the step, [pass][gemm] in us.
+def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, trials: int = 10):
+    """Device time of one launch of each GEMM of the step, [pass][gemm] in us:
+    the median and the best of `trials` trials.
 
     Each GEMM is timed as a CUDA graph of `launches` back-to-back launches on one
     stream, rotating through enough copies of its weights to exceed 4x the L2
-    cache (so no launch finds its weights in L2), with CUDA events around the
-    whole graph on the launching stream.  No event sits between the launches
-    (an event-record node in a graph costs several microseconds)."""
+    cache (so no launch finds its weights in L2); a trial is `replays` replays
+    of that graph between CUDA events on the launching stream, divided by the
+    launches it ran.  No event sits between the launches (an event-record node
+    in a graph costs several microseconds)."""
     import torch
 
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
     out = np.zeros((len(PASSES), len(si.MIXED_LAYER)))
+    best = np.zeros_like(out)
     stream = torch.cuda.Stream()
     for i, spec in enumerate(si.MIXED_LAYER):
         base = weights[0][i]
@@ -290,17 +305,21 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3):
             g.replay()
             g.replay()
             torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(replays):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            out[pi, i] = 1e3 * e0.elapsed_time(e1) / (replays * launches)
+            t = []
+            for _ in range(trials):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(replays):
+                    g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                t.append(1e3 * e0.elapsed_time(e1) / (replays * launches))
+            out[pi, i] = float(np.median(t))
+            best[pi, i] = float(np.min(t))
             del g
         del copies
     torch.cuda.empty_cache()
-    return out
+    return out, best
 
 
 def _random_packed_copies(dev, N, K, gen):
@@ -322,9 +341,10 @@ def _random_packed_copies(dev, N, K, gen):
     return copies, nbytes
 
 
-def _graph_us(one, n_copy, launches, replays):
-    """Average device time of one launch: a CUDA graph of back-to-back launches
-    rotating over the weight copies, CUDA events around the replays."""
+def _graph_us(one, n_copy, launches, replays, trials: int = 10):
+    """Device time of one launch, median over `trials`: a CUDA graph of
+    back-to-back launches rotating over the weight copies, CUDA events around
+    each trial's replays."""
     import torch
 
     stream = torch.cuda.Stream()
@@ -338,14 +358,17 @@ def _graph_us(one, n_copy, launches, replays):
             one(r % n_copy)
     g.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(replays):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
+    t = []
+    for _ in range(trials):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t.append(1e3 * e0.elapsed_time(e1) / (replays * launches))
     del g
-    return 1e3 * e0.elapsed_time(e1) / (replays * launches)
+    return float(np.median(t))
 
 
 def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
@@ -500,20 +523,29 @@ def oracle_sample_frac(target_s: float, threads: int) -> float:
     return frac
 
 
-def cpu_baseline(target_s: float = 12.0):
-    import oracle
-
-    threads = oracle.default_threads()
+def _timed_oracle(target_s: float, threads: int):
     frac = oracle_sample_frac(target_s, threads)
     items = _oracle_inputs(frac)
     t, reps = 0.0, 0
     while t < 0.8 * target_s or reps == 0:   # the whole workload may take less than target_s
         t += _oracle_run(items, threads)
         reps += 1
-    return {"value": round(reps * _oracle_bytes(items) / t / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle",
+    return reps * _oracle_bytes(items) / t / 1e9, frac, reps, t
+
+
+def cpu_baseline(target_s: float = 12.0, single_core_s: float = 6.0):
+    """The float64 oracle on every host core, and on one core."""
+    import oracle
+
+    threads = oracle.default_threads()
+    value, frac, reps, t = _timed_oracle(target_s, threads)
+    one, frac1, reps1, t1 = _timed_oracle(single_core_s, 1)
+    return {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": "float64 C oracle, %d threads, on the first %.3f%% of the rows of each of the 5 GEMMs of %s at "
-                      "M=1 and M=8 (same byte formula), %d pass(es), %.1f s" % (threads, 100 * frac, WORKLOAD, reps, t)}
+                      "M=1 and M=8 (same byte formula), %d pass(es), %.1f s" % (threads, 100 * frac, WORKLOAD, reps, t),
+            "single_core": {"value": round(one, 4), "unit": "GB/s", "cores": 1,
+                            "sample": "the same oracle on 1 thread, first %.3f%% of the rows, %d pass(es), %.1f s"
+                                      % (100 * frac1, reps1, t1)}}
 
 
 def reference_arm(args):
@@ -536,7 +568,7 @@ def reference_arm(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "sample_rows_frac": frac},
+            "config": bench_config(args.gpus),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": "float64 C oracle on the first %.3f%% of the rows of each GEMM of %s "
                                        "at M=1 and M=8" % (100 * frac, WORKLOAD)},
@@ -623,7 +655,7 @@ def main(argv=None):
     sampler = ClockSampler(local)
     # Per-launch device time of each GEMM (CUDA events around graphs of
     # back-to-back launches); this also brings the GPU to its loaded clocks.
-    dur_us = per_launch_us(weights, xs, ys, ws)
+    dur_us, best_us = per_launch_us(weights, xs, ys, ws)
     fused = fused_epilogues_us(dev)
 
     for i in range(args.warmup):
@@ -659,7 +691,8 @@ def main(argv=None):
             b = gemm_bytes(spec, M)
             d = float(dur_us[pi, i])
             per.append({"gemm": spec.name, "fmt": spec.fmt, "M": M, "N": spec.N, "K": spec.K,
-                        "us": round(d, 3), "GB/s": round(b / d / 1e3, 1), "frac": round(b / d / 1e3 / peak, 4)})
+                        "us": round(d, 3), "us_best": round(float(best_us[pi, i]), 3),
+                        "GB/s": round(b / d / 1e3, 1), "frac": round(b / d / 1e3 / peak, 4)})
             if spec.fmt == "nvfp4":
                 nv_bytes += b
                 nv_us += d
@@ -671,13 +704,7 @@ def main(argv=None):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD,
-                   "gemms": ["%s %s %dx%d" % (s.name, s.fmt, s.N, s.K) for s in si.MIXED_LAYER],
-                   "M": list(PASSES), "operands": "NVFP4/FP8 weights x FP16 activations, FP32 accumulation",
-                   "l2": "inputs larger than L2: %d rotating weight copies, %.0f MB" %
-                         (COPIES, COPIES * sum(weight_bytes(s) for s in si.MIXED_LAYER) / 1e6),
-                   "bytes_per_step": sb, "launch": "CUDA graph per step", "parallelism": "replicas" if world > 1
-                   else "single GPU"},
+        "config": bench_config(world),
         "frac_of_peak": round(value / world / peak, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,

@@ -32,9 +32,16 @@ OUT_F32 = 1
 FMT_NVFP4 = 0
 FMT_FP8 = 1
 MAX_M = 8
+MAX_GROUP = 8
 
 _lock = threading.Lock()
 _lib = None
+
+
+class GroupMember(ctypes.Structure):
+    """skinny_nvfp4_group_member of include/skinny.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("w_packed", ctypes.c_void_p), ("global_scale", ctypes.c_float),
+                ("N", ctypes.c_int64), ("y", ctypes.c_void_p)]
 
 
 class SkinnyError(RuntimeError):
@@ -80,6 +87,9 @@ def library() -> ctypes.CDLL:
                 "skinny_nvfp4_gemm_silu_mul": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
                                                               ctypes.c_int, p, sz, p]),
                 "skinny_static_workspace_capacity": (sz, []),
+                "skinny_nvfp4_gemm_grouped": (ctypes.c_int, [ctypes.POINTER(GroupMember), ctypes.c_int,
+                                                             ctypes.c_int, i64, ctypes.c_int, p, sz, p]),
+                "skinny_debug_static_workspace_address": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p)]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(lib, name)
@@ -279,6 +289,31 @@ def gemm_add_into(y, x, w, residual, workspace=None, stream=None) -> None:
         st = lib.skinny_fp8_gemm_add(x.data_ptr(), M, K, w.codes.data_ptr(), w.channel_scale.data_ptr(), w.N,
                                      residual.data_ptr(), y.data_ptr(), out, ws_ptr, ws_bytes, h)
         _check(st, "skinny_fp8_gemm_add")
+
+
+def gemm_grouped_into(ys, xs, ws, workspace=None, stream=None) -> None:
+    """ys[i][M, N_i] = xs[i][M, K] . W_i^T for every i, in ONE launch (NVFP4
+    weights of the same K; ys all float16 or all float32, preallocated)."""
+    import torch
+
+    if not (len(ys) == len(xs) == len(ws)) or not 1 <= len(ws) <= MAX_GROUP:
+        raise ValueError("ys, xs and ws must have the same length, 1..%d" % MAX_GROUP)
+    M, K = xs[0].shape
+    dt = ys[0].dtype
+    members = (GroupMember * len(ws))()
+    for i, (y, x, w) in enumerate(zip(ys, xs, ws)):
+        if w.fmt != FMT_NVFP4 or w.K != K:
+            raise ValueError("grouped GEMMs take NVFP4 weights of one K")
+        if x.dtype != torch.float16 or not x.is_contiguous() or x.shape != (M, K):
+            raise ValueError("every x must be a contiguous float16 [%d, %d] tensor" % (M, K))
+        if y.shape != (M, w.N) or not y.is_contiguous() or y.dtype != dt or dt not in (torch.float16, torch.float32):
+            raise ValueError("every y must be a contiguous [M, N_i] tensor of one dtype (float16 or float32)")
+        members[i] = GroupMember(x.data_ptr(), w.data.data_ptr(), w.global_scale, w.N, y.data_ptr())
+    out = OUT_F32 if dt == torch.float32 else OUT_F16
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = library().skinny_nvfp4_gemm_grouped(members, len(ws), M, K, out, ws_ptr, ws_bytes, _stream_handle(stream))
+    _check(st, "skinny_nvfp4_gemm_grouped")
 
 
 def gemm(x, w, out_dtype=None, workspace=None, stream=None):

@@ -128,15 +128,26 @@ struct Smem {
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
-struct Params {
+// One GEMM of a launch.  A launch runs one GEMM, or a group of independent
+// GEMMs of the same K (and M, format and output type) whose row tiles are
+// concatenated into one tile sequence: member m owns row tiles
+// [g_begin, next member's g_begin).
+struct Member {
     const uint16_t* x;            // [M][K] fp16 bits
     const uint8_t* codes;         // packed tiles (NVFP4 tiles carry their block scales)
     const float* channel_scale;   // FP8 per-output-channel scale [N]
     void* y;                      // [M][N]
     const void* residual;         // [M][N], y's dtype, added before the output rounding (or null; may alias y)
-    uint2* partials;              // [P][16 warps][32 lanes] encoded float pairs (split-K only)
     float out_scale;              // NVFP4 per-tensor scale (FP8: unused, the channel scales apply)
-    int M, K, N;
+    int N;
+    int g_begin;                  // first row tile of this GEMM in the launch's tile sequence
+};
+
+struct Params {
+    Member mem[SKINNY_MAX_GROUP];
+    int n_members;
+    uint2* partials;              // [P][16 warps][32 lanes] encoded float pairs (split-K only)
+    int M, K;
     int C;                        // K tiles per row tile
     int U;                        // tiles in total (G * C)
     int Q;                        // scheduling quantum: 1 (split K) or C (whole row tiles)
@@ -151,6 +162,14 @@ struct Params {
     int* out_idx;                 // [M]
     float* out_val;               // [M]
 };
+
+// The GEMM of the launch that owns row tile g.
+__device__ __forceinline__ int member_of(const Params& p, int g)
+{
+    int m = p.n_members - 1;
+    while (m > 0 && g < p.mem[m].g_begin) --m;
+    return m;
+}
 
 // CTA b of P takes quanta [b*UQ/P, (b+1)*UQ/P) of the UQ = U/Q quanta.
 __host__ __device__ __forceinline__ int range_start(int b, int P, int UQ, int Q)
@@ -228,8 +247,9 @@ template <int FMT>
 __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane)
 {
     const int gid = lane >> 2, t = lane & 3;
-    const int n = g * kTileRows + strip * kStripRows + gid + 8 * h;
-    const float sc = (FMT == SKINNY_FMT_NVFP4) ? p.out_scale : (n < p.N ? p.channel_scale[n] : 0.f);
+    const Member& mb = p.mem[member_of(p, g)];
+    const int n = (g - mb.g_begin) * kTileRows + strip * kStripRows + gid + 8 * h;
+    const float sc = (FMT == SKINNY_FMT_NVFP4) ? mb.out_scale : (n < mb.N ? mb.channel_scale[n] : 0.f);
     if (p.argmax) {
         // The warp's best (value, row) per token: lanes with the same t hold
         // the same two tokens for eight rows; one shared-memory atomic per
@@ -238,7 +258,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int m = 2 * t + e;
-            unsigned long long key = (n < p.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
+            unsigned long long key = (n < mb.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
 #pragma unroll
             for (int d = 4; d < 32; d <<= 1) {
                 const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, d);
@@ -248,25 +268,25 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
         }
         return;
     }
-    if (n >= p.N) return;
+    if (n >= mb.N) return;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int m = 2 * t + e;
         if (m >= p.M) continue;
-        const size_t idx = (size_t)m * p.N + n;
+        const size_t idx = (size_t)m * mb.N + n;
         // Rounded FP32 product, never contracted with the add below, so the
         // fused add sees exactly the value the plain GEMM stores.
         float val = __fmul_rn(v[e], sc);
         // Fused residual add: one FP32 add, then the single output rounding.
         // Each element is read and written by this thread only, so the
         // residual may be y itself.
-        if (p.residual)
-            val = __fadd_rn(val, p.out_f32 ? static_cast<const float*>(p.residual)[idx]
-                                           : __half2float(static_cast<const __half*>(p.residual)[idx]));
+        if (mb.residual)
+            val = __fadd_rn(val, p.out_f32 ? static_cast<const float*>(mb.residual)[idx]
+                                           : __half2float(static_cast<const __half*>(mb.residual)[idx]));
         if (p.out_f32)
-            static_cast<float*>(p.y)[idx] = val;
+            static_cast<float*>(mb.y)[idx] = val;
         else
-            static_cast<__half*>(p.y)[idx] = __float2half_rn(val);
+            static_cast<__half*>(mb.y)[idx] = __float2half_rn(val);
     }
 }
 
@@ -282,19 +302,20 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[2], int g, i
     const int gid = lane >> 2, t = lane & 3;
     const int r = strip * kStripRows + gid + 8 * h;
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
-    act[r * SKINNY_MAX_M + 2 * t] = v[0] * p.out_scale;
-    act[r * SKINNY_MAX_M + 2 * t + 1] = v[1] * p.out_scale;
+    const Member& mb = p.mem[0];   // the fused SiLU*mul runs one GEMM per launch
+    act[r * SKINNY_MAX_M + 2 * t] = v[0] * mb.out_scale;
+    act[r * SKINNY_MAX_M + 2 * t + 1] = v[1] * mb.out_scale;
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
     const int jl = threadIdx.x % 64, m = threadIdx.x / 64;          // 64 outputs x 8 tokens
-    const int F = p.N / 2, j = g * 64 + jl;
+    const int F = mb.N / 2, j = g * 64 + jl;
     if (m < p.M && j < F) {
         const float gate = act[jl * SKINNY_MAX_M + m], up = act[(64 + jl) * SKINNY_MAX_M + m];
         const float val = gate / (1.f + expf(-gate)) * up;
         const size_t idx = (size_t)m * F + j;
         if (p.out_f32)
-            static_cast<float*>(p.y)[idx] = val;
+            static_cast<float*>(mb.y)[idx] = val;
         else
-            static_cast<__half*>(p.y)[idx] = __float2half_rn(val);
+            static_cast<__half*>(mb.y)[idx] = __float2half_rn(val);
     }
 }
 
@@ -397,9 +418,10 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_fi
 template <int FMT>
 __device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int u)
 {
+    const Member& mb = p.mem[member_of(p, u / p.C)];
+    const uint8_t* src = mb.codes + (size_t)(u - mb.g_begin * p.C) * Tile<FMT>::kBytes;
     ptx::mbar_arrive_expect_tx(&full[s], Tile<FMT>::kBytes);
-    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, p.codes + (size_t)u * Tile<FMT>::kBytes, Tile<FMT>::kBytes,
-                  &full[s], ptx::policy_evict_first());
+    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, src, Tile<FMT>::kBytes, &full[s], ptx::policy_evict_first());
 }
 
 // The B fragments of one K tile for this lane: token gid (row xrow of x),
@@ -530,15 +552,19 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 16;
         w.lane_scale = 0;
     }
-    // Activations: token gid, columns c*512 + (2kq + u)*64 + [16t, 16t+16).
+    // Activations: token gid, columns c*512 + (2kq + u)*64 + [16t, 16t+16),
+    // from the x of the GEMM that owns the tile.
     const bool xvalid = gid < p.M;
-    const uint16_t* xrow = p.x + (size_t)(xvalid ? gid : 0) * p.K;
+    const size_t xoff = (size_t)(xvalid ? gid : 0) * p.K;
     const int kb_lane = 2 * kq * kChunkK + 16 * t;
 
     // The range is walked from its last tile down to its first.
     int cur_g = sc.last_g, parity = 0;
     int g = sc.last_g, c = sc.u_last - sc.last_g * p.C;   // tile being processed
     int nc = c;                                            // K tile whose activations are fetched next
+    int ng = g;                                            // ... and its row tile
+    int nm = member_of(p, ng);                             // ... and its GEMM
+    const uint16_t* xrow = p.mem[nm].x + xoff;
     const uint32_t smem32 = ptx::smem_addr(smem);
     int* released = reinterpret_cast<int*>(smem + S::kCountOff);
     // Contributors of a row tile: only the two at the ends of the range are shared.
@@ -561,7 +587,11 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     // One tile per iteration; the body is written for buffer B = i & 1 (the
     // loop is unrolled by two so the ping-pong buffers stay in registers).
     auto step = [&](int i, uint32_t (&cur)[2][8], uint32_t (&nxt)[2][8]) {
-        nc = (nc == 0 ? p.C : nc) - 1;
+        if (nc == 0) {
+            nc = p.C;
+            if (--ng < p.mem[nm].g_begin && nm > 0) xrow = p.mem[--nm].x + xoff;
+        }
+        --nc;
         if (i + 1 < n_units) {   // next tile's activations, one tile ahead
             load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, nxt[0]);
             load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, nxt[1]);
@@ -718,12 +748,13 @@ struct Plan {
     size_t partial_bytes, workspace_bytes;
 };
 
-static int make_plan(int fmt, int64_t N, int64_t K, int sms, bool split, Plan* pl)
+static int64_t row_tiles(int64_t N) { return (N + kTileRows - 1) / kTileRows; }
+
+// G row tiles (all GEMMs of the launch together) of K columns each.
+static int make_plan(int64_t G, int64_t K, int sms, bool split, Plan* pl)
 {
-    const int64_t G = (N + kTileRows - 1) / kTileRows;
-    (void)fmt;
     const int64_t C = (K + kTileK - 1) / kTileK;
-    if (G * C >= (int64_t(1) << 31)) return SKINNY_ERR_UNSUPPORTED;
+    if (G <= 0 || G * C >= (int64_t(1) << 31)) return SKINNY_ERR_UNSUPPORTED;
     pl->G = (int)G;
     pl->C = (int)C;
     pl->U = (int)(G * C);
@@ -748,15 +779,37 @@ static int check_common(const void* x, int M, int64_t K, int64_t N, const void* 
     return SKINNY_OK;
 }
 
+// A launch of one GEMM: member 0 only.
+static Params single(const void* x, int M, int64_t K, const void* w_packed, const float* channel_scale,
+                     float out_scale, int64_t N, void* y, const void* residual, int out_dtype)
+{
+    Params p{};
+    p.n_members = 1;
+    Member& mb = p.mem[0];
+    mb.x = static_cast<const uint16_t*>(x);
+    mb.codes = static_cast<const uint8_t*>(w_packed);
+    mb.channel_scale = channel_scale;
+    mb.y = y;
+    mb.residual = residual;
+    mb.out_scale = out_scale;
+    mb.N = (int)N;
+    mb.g_begin = 0;
+    p.M = M;
+    p.K = (int)K;
+    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    return p;
+}
+
+// Launch the GEMM(s) of p, whose members' row tiles add up to G.
 template <int FMT>
-static int launch(Params p, int64_t N, int64_t K, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+static int launch(Params p, int64_t G, int64_t K, void* workspace, size_t workspace_bytes, cudaStream_t stream)
 {
     int sms = 0;
     int rc = current_device(&sms);
     if (rc != SKINNY_OK) return rc;
     const bool split = workspace != nullptr;
     Plan pl;
-    rc = make_plan(FMT, N, K, sms, split, &pl);
+    rc = make_plan(G, K, sms, split, &pl);
     if (rc != SKINNY_OK) return rc;
     if (split && workspace_bytes < pl.workspace_bytes) return SKINNY_ERR_WORKSPACE;
     p.C = pl.C;
@@ -802,7 +855,7 @@ extern "C" const char* skinny_status_string(int status)
     }
 }
 
-extern "C" int skinny_version(void) { return 100; }
+extern "C" int skinny_version(void) { return 101; }
 
 extern "C" int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes)
 {
@@ -813,7 +866,7 @@ extern "C" int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size
     int rc = current_device(&sms);
     if (rc != SKINNY_OK) return rc;
     Plan pl;
-    rc = make_plan(fmt, N, K, sms, true, &pl);
+    rc = make_plan(row_tiles(N), K, sms, true, &pl);
     if (rc != SKINNY_OK) return rc;
     *bytes = pl.workspace_bytes;
     return SKINNY_OK;
@@ -826,7 +879,7 @@ extern "C" int skinny_debug_schedule(int64_t N, int64_t K, int sms, int split, i
 {
     if (!out || !ctas || sms <= 0 || N <= 0 || K <= 0 || K % 16 != 0) return SKINNY_ERR_INVALID_ARG;
     Plan pl;
-    const int rc = make_plan(SKINNY_FMT_NVFP4, N, K, sms, split != 0, &pl);
+    const int rc = make_plan(row_tiles(N), K, sms, split != 0, &pl);
     if (rc != SKINNY_OK) return rc;
     *ctas = pl.P;
     if (pl.P > cap) return SKINNY_ERR_WORKSPACE;
@@ -855,16 +908,8 @@ extern "C" int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_
     if (rc != SKINNY_OK) return rc;
     if (!w_packed) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.y = y;
-    p.out_scale = global_scale;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)N;
-    p.out_f32 = out_dtype == SKINNY_OUT_F32;
-    return launch<SKINNY_FMT_NVFP4>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    const Params p = single(x, M, K, w_packed, nullptr, global_scale, N, y, nullptr, out_dtype);
+    return launch<SKINNY_FMT_NVFP4>(p, row_tiles(N), K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_packed, const float* channel_scale,
@@ -875,17 +920,8 @@ extern "C" int skinny_fp8_gemm(const void* x, int M, int64_t K, const void* w_pa
     if (rc != SKINNY_OK) return rc;
     if (!w_packed || !channel_scale) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16) || !aligned(channel_scale, 4)) return SKINNY_ERR_ALIGNMENT;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.channel_scale = channel_scale;
-    p.y = y;
-    p.out_scale = 1.0f;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)N;
-    p.out_f32 = out_dtype == SKINNY_OUT_F32;
-    return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    const Params p = single(x, M, K, w_packed, channel_scale, 1.0f, N, y, nullptr, out_dtype);
+    return launch<SKINNY_FMT_FP8>(p, row_tiles(N), K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_nvfp4_gemm_add(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
@@ -898,17 +934,8 @@ extern "C" int skinny_nvfp4_gemm_add(const void* x, int M, int64_t K, const void
     if (rc != SKINNY_OK) return rc;
     if (!w_packed) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.y = y;
-    p.residual = residual;
-    p.out_scale = global_scale;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)N;
-    p.out_f32 = out_dtype == SKINNY_OUT_F32;
-    return launch<SKINNY_FMT_NVFP4>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    const Params p = single(x, M, K, w_packed, nullptr, global_scale, N, y, residual, out_dtype);
+    return launch<SKINNY_FMT_NVFP4>(p, row_tiles(N), K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_fp8_gemm_add(const void* x, int M, int64_t K, const void* w_packed, const float* channel_scale,
@@ -921,18 +948,8 @@ extern "C" int skinny_fp8_gemm_add(const void* x, int M, int64_t K, const void* 
     if (rc != SKINNY_OK) return rc;
     if (!w_packed || !channel_scale) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16) || !aligned(channel_scale, 4)) return SKINNY_ERR_ALIGNMENT;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.channel_scale = channel_scale;
-    p.y = y;
-    p.residual = residual;
-    p.out_scale = 1.0f;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)N;
-    p.out_f32 = out_dtype == SKINNY_OUT_F32;
-    return launch<SKINNY_FMT_FP8>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    const Params p = single(x, M, K, w_packed, channel_scale, 1.0f, N, y, residual, out_dtype);
+    return launch<SKINNY_FMT_FP8>(p, row_tiles(N), K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_nvfp4_gemm_silu_mul(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
@@ -944,17 +961,10 @@ extern "C" int skinny_nvfp4_gemm_silu_mul(const void* x, int M, int64_t K, const
     if (rc != SKINNY_OK) return rc;
     if (!w_packed) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.y = y;
-    p.out_scale = global_scale;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)(2 * F);
-    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    Params p = single(x, M, K, w_packed, nullptr, global_scale, 2 * F, y, nullptr, out_dtype);
     p.silu_mul = 1;
-    return launch<SKINNY_FMT_NVFP4>(p, 2 * F, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    return launch<SKINNY_FMT_NVFP4>(p, row_tiles(2 * F), K, workspace, workspace_bytes,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_packed, float global_scale,
@@ -966,18 +976,41 @@ extern "C" int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const v
     if (!w_packed || !argmax_idx) return SKINNY_ERR_INVALID_ARG;
     if (!aligned(w_packed, 16) || !aligned(argmax_idx, 4)) return SKINNY_ERR_ALIGNMENT;
     if (!workspace) return SKINNY_ERR_WORKSPACE;
-    Params p{};
-    p.x = static_cast<const uint16_t*>(x);
-    p.codes = static_cast<const uint8_t*>(w_packed);
-    p.out_scale = global_scale;
-    p.M = M;
-    p.K = (int)K;
-    p.N = (int)N;
-    p.out_f32 = 1;
+    Params p = single(x, M, K, w_packed, nullptr, global_scale, N, nullptr, nullptr, SKINNY_OUT_F32);
     p.argmax = 1;
     p.out_idx = argmax_idx;
     p.out_val = argmax_val;
-    return launch<SKINNY_FMT_NVFP4>(p, N, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    return launch<SKINNY_FMT_NVFP4>(p, row_tiles(N), K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int skinny_nvfp4_gemm_grouped(const skinny_nvfp4_group_member* members, int count, int M, int64_t K,
+                                         int out_dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!members || count < 1) return SKINNY_ERR_INVALID_ARG;
+    if (count > SKINNY_MAX_GROUP) return SKINNY_ERR_UNSUPPORTED;
+    Params p{};
+    int64_t G = 0;
+    for (int m = 0; m < count; ++m) {
+        const skinny_nvfp4_group_member& in = members[m];
+        const int rc = check_common(in.x, M, K, in.N, in.y, out_dtype, workspace);
+        if (rc != SKINNY_OK) return rc;
+        if (!in.w_packed) return SKINNY_ERR_INVALID_ARG;
+        if (!aligned(in.w_packed, 16)) return SKINNY_ERR_ALIGNMENT;
+        Member& mb = p.mem[m];
+        mb.x = static_cast<const uint16_t*>(in.x);
+        mb.codes = static_cast<const uint8_t*>(in.w_packed);
+        mb.y = in.y;
+        mb.out_scale = in.global_scale;
+        mb.N = (int)in.N;
+        mb.g_begin = (int)G;
+        G += row_tiles(in.N);
+        if (G >= (int64_t(1) << 30)) return SKINNY_ERR_UNSUPPORTED;
+    }
+    p.n_members = count;
+    p.M = M;
+    p.K = (int)K;
+    p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    return launch<SKINNY_FMT_NVFP4>(p, G, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -1026,7 +1059,7 @@ extern "C" int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, cons
     rc = current_device(&sms);
     if (rc != SKINNY_OK) return rc;
     Plan pl;
-    rc = make_plan(SKINNY_FMT_NVFP4, N, K, sms, true, &pl);
+    rc = make_plan(row_tiles(N), K, sms, true, &pl);
     if (rc != SKINNY_OK) return rc;
     if (pl.workspace_bytes > kStaticWorkspaceBytes) return SKINNY_ERR_UNSUPPORTED;
     void* ws = nullptr;
@@ -1038,6 +1071,14 @@ extern "C" int skinny_nvfp4_gemm_static_ws(const void* x, int M, int64_t K, cons
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, pl.workspace_bytes, st) != cudaSuccess) return SKINNY_ERR_CUDA;
     return skinny_nvfp4_gemm(x, M, K, w_packed, global_scale, N, y, out_dtype, ws, kStaticWorkspaceBytes, stream);
+}
+
+// Test hook: the device address of the static scratch array on the current
+// device (the same lookup skinny_nvfp4_gemm_static_ws makes).
+extern "C" int skinny_debug_static_workspace_address(void** addr)
+{
+    if (!addr) return SKINNY_ERR_INVALID_ARG;
+    return static_workspace_address(addr);
 }
 
 extern "C" int skinny_device_error(int clear, unsigned* flags)

@@ -33,7 +33,12 @@ def gather_columns(y_local, N: int, group=None):
     """All-gather the ranks' column blocks y[:, start_r:stop_r] (each [M, width_r],
     same dtype and device) into the full y [M, N] on every rank.  Blocks may
     differ in width (the last shard is ragged); they travel padded to the widest
-    one and are trimmed back in rank order."""
+    one and are trimmed back in rank order.
+
+    Device tensors are gathered in the order of torch's current stream (NCCL
+    waits on it).  A gloo group moves host tensors only, so device blocks are
+    staged through host memory there and the result is returned on y_local's
+    device."""
     import torch
     import torch.distributed as dist
 
@@ -43,29 +48,41 @@ def gather_columns(y_local, N: int, group=None):
     rank = dist.get_rank(group)
     if y_local.shape[1] != widths[rank]:
         raise ValueError("y_local must hold this rank's %d columns" % widths[rank])
+    staged = y_local.is_cuda and dist.get_backend(group) == "gloo"
+    where = torch.device("cpu") if staged else y_local.device
     w_max = max(widths)
-    send = torch.zeros((M, w_max), dtype=y_local.dtype, device=y_local.device)
+    send = torch.zeros((M, w_max), dtype=y_local.dtype, device=where)
     send[:, :widths[rank]] = y_local
-    recv = [torch.empty((M, w_max), dtype=y_local.dtype, device=y_local.device) for _ in range(world)]
+    recv = [torch.empty((M, w_max), dtype=y_local.dtype, device=where) for _ in range(world)]
     dist.all_gather(recv, send, group=group)
-    return torch.cat([recv[r][:, :widths[r]] for r in range(world)], dim=1)
+    y = torch.cat([recv[r][:, :widths[r]] for r in range(world)], dim=1)
+    return y.to(y_local.device) if staged else y
 
 
 def column_parallel_gemm(x, w_shard, N: int, group=None, out_dtype=None, workspace=None, stream=None):
     """y [M, N] = x . W^T on every rank, each rank holding the packed rows
-    shard_rows(N, world, rank) of W as `w_shard` (PackedNVFP4 or PackedFP8)."""
+    shard_rows(N, world, rank) of W as `w_shard` (PackedNVFP4 or PackedFP8).
+
+    With `stream` given, the local GEMM, the staging copies and the all-gather
+    are all issued on that stream (torch's current stream is switched to it for
+    the call), so the gather reads the GEMM's output only after the kernel has
+    written it; x must be ready in that stream's order, and the returned y is
+    ready in it too.  Without `stream`, everything runs on the current stream."""
+    import contextlib
+
+    import torch
     import torch.distributed as dist
 
     from . import gemm
 
     world, rank = dist.get_world_size(group), dist.get_rank(group)
     start, stop = shard_rows(N, world, rank)
-    if stop == start:   # N < world * 128: this rank owns no rows
-        import torch
-
-        y_local = torch.empty((x.shape[0], 0), dtype=out_dtype or torch.float16, device=x.device)
-    else:
-        if w_shard is None or w_shard.N != stop - start:
-            raise ValueError("w_shard must hold rows [%d, %d) of W" % (start, stop))
-        y_local = gemm(x, w_shard, out_dtype=out_dtype, workspace=workspace, stream=stream)
-    return gather_columns(y_local, N, group)
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with ctx:
+        if stop == start:   # N < world * 128: this rank owns no rows
+            y_local = torch.empty((x.shape[0], 0), dtype=out_dtype or torch.float16, device=x.device)
+        else:
+            if w_shard is None or w_shard.N != stop - start:
+                raise ValueError("w_shard must hold rows [%d, %d) of W" % (start, stop))
+            y_local = gemm(x, w_shard, out_dtype=out_dtype, workspace=workspace)
+        return gather_columns(y_local, N, group)

@@ -70,6 +70,9 @@ typedef enum { SKINNY_FMT_NVFP4 = 0, SKINNY_FMT_FP8 = 1 } skinny_format;
 
 #define SKINNY_MAX_M 8
 
+/* Most GEMMs one skinny_nvfp4_gemm_grouped call can run. */
+#define SKINNY_MAX_GROUP 8
+
 /* Name of a skinny_status value ("SKINNY_OK", ...); never NULL. */
 const char* skinny_status_string(int status);
 
@@ -136,11 +139,24 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
  * skinny_device_error(), zero-fill it again.  Its layout is the same for
  * every shape on a device, so one workspace serves calls of any shape in
  * turn; it must not be shared by calls that can run at the same time.
+ * Residency: with a workspace, the CTA that finishes a row tile waits
+ * (bounded, 1 s) for the partial sums of lower-numbered CTAs of the same
+ * grid.  The grid has at most one CTA per SM and the wait ends as soon as
+ * those CTAs have run, so it assumes that they can run: the whole GPU, or
+ * CTAs dispatched in increasing order.  Where the GPU is shared so that only
+ * part of the grid can be resident (an MPS client limited to fewer SMs than
+ * the device has, say), pass no workspace: the whole-tile schedule has no
+ * wait between CTAs.
  * Returns SKINNY_OK and *bytes, or SKINNY_ERR_INVALID_ARG / _UNSUPPORTED /
  * _CUDA. */
 int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
 
 /* NVFP4 weight-only GEMM: y = x . W^T with W from skinny_pack_nvfp4.
+ * This is the "QPN2" operation of the v100-skinny pages (taozi.news article,
+ * section "自研 QPN 内核": NVFP4 weights stay 4-bit on their way out of HBM
+ * and become FP16 in registers, against FP16 activations; M=1 is one decode
+ * token and M=8 the k=7 verify round; aiwitness.kr post, section
+ * "내가 실제로 만든 것").
  *   x            device [M][K] FP16, 16-byte aligned, read-only during the call.
  *   M            1..8 (rows of x: tokens of one decode / verify round).
  *   K            multiple of 16.
@@ -161,6 +177,10 @@ int skinny_nvfp4_gemm(const void* x, int M, int64_t K, const void* w_packed, flo
                       void* y, int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /* FP8 (E4M3) weight-only GEMM with a per-output-channel FP32 scale.
+ * This is the "QPN8" operation that serves the checkpoint's FP8 regions
+ * (taozi.news article, section "v1.1 的关键改进": FP4 regions stay FP4 and
+ * FP8 regions stay FP8, with FP16 activations; its M=1..4 bandwidth is quoted
+ * in section "自研 QPN 内核").
  *   w_packed       device, from skinny_pack_fp8, 16-byte aligned.
  *   channel_scale  device float[N], 4-byte aligned.
  * Other arguments as skinny_nvfp4_gemm (workspace sized with SKINNY_FMT_FP8). */
@@ -229,6 +249,36 @@ int skinny_nvfp4_gemm_argmax(const void* x, int M, int64_t K, const void* w_pack
                              int32_t* argmax_idx, float* argmax_val, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* One GEMM of a grouped launch (see skinny_nvfp4_gemm_grouped).  Plain
+ * pointers; the struct is read on the host during the call. */
+typedef struct {
+    const void* x;         /* device [M][K] FP16, 16-byte aligned */
+    const void* w_packed;  /* device, from skinny_pack_nvfp4 with this N and the call's K, 16-byte aligned */
+    float global_scale;    /* FP32 per-tensor scale */
+    int64_t N;             /* output features of this GEMM */
+    void* y;               /* device [M][N], FP16 or FP32 per the call's out_dtype, 4-byte aligned */
+} skinny_nvfp4_group_member;
+
+/* Several independent NVFP4 GEMMs of the same K, M and output type in ONE
+ * launch: y_i = x_i . W_i^T for i < count.  The attention projections of a
+ * decoder layer (the 5120-wide q, k/v and o shapes the v100-skinny pages
+ * measure: taozi.news article, section "自研 QPN 内核") each stream only
+ * ~15 MB, too little to amortise a launch's ramp-up and tail on their own;
+ * their row tiles are concatenated into one tile sequence that the stream-K
+ * schedule spreads over all SMs, so the fixed cost is paid once.  Members
+ * may share x (q, k and v read the same activations) but their y must not
+ * overlap each other or any x.  Each y_i is exactly what skinny_nvfp4_gemm
+ * computes for member i up to FP32 summation order (the split points of K
+ * differ); the order is fixed for a given member list, so results are
+ * bitwise reproducible.
+ *   members    host array of `count` entries.
+ *   count      1..SKINNY_MAX_GROUP (more: UNSUPPORTED; 0 or null: INVALID_ARG).
+ *   workspace  optional, as for skinny_nvfp4_gemm (same size: it depends on
+ *              the device only).
+ * Errors: per member as skinny_nvfp4_gemm. */
+int skinny_nvfp4_gemm_grouped(const skinny_nvfp4_group_member* members, int count, int M, int64_t K,
+                              int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* NVFP4 GEMM for callers that cannot allocate device memory.
  *
  * There is no counterpart of this entry point on the v100-skinny pages; it
@@ -269,6 +319,12 @@ int skinny_debug_schedule(int64_t N, int64_t K, int sms, int split, int* out, in
 
 /* Size in bytes of the static scratch array used by skinny_nvfp4_gemm_static_ws. */
 size_t skinny_static_workspace_capacity(void);
+
+/* Test hook: *addr receives the device address of that static array on the
+ * current device (looked up with cudaGetSymbolAddress, as the entry point
+ * does), so that a test can overwrite it between calls.  Returns SKINNY_OK,
+ * SKINNY_ERR_INVALID_ARG (null addr) or SKINNY_ERR_CUDA. */
+int skinny_debug_static_workspace_address(void** addr);
 
 /* Device-side error word of the current device.  Every wait inside the
  * kernels is bounded; a wait that gives up sets a bit here instead of

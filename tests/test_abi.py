@@ -174,3 +174,39 @@ def test_library_sources_allocate_no_device_memory():
         assert not calls.search(code), (name, calls.search(code).group(0))
     skinny_cu = open(os.path.join(csrc, "skinny.cu")).read()
     assert len(re.findall(r"static __device__ __align__\(256\) unsigned char g_static_workspace", skinny_cu)) == 1
+
+
+def _group(n, **kw):
+    a = dict(x=ALIGNED, w=ALIGNED, g=1.0, N=256, y=ALIGNED)
+    a.update(kw)
+    arr = (sk.GroupMember * max(n, 1))()
+    for i in range(n):
+        arr[i] = sk.GroupMember(a["x"], a["w"], a["g"], a["N"], a["y"])
+    return arr
+
+
+@pytest.mark.parametrize("count,kw,status", [
+    (0, {}, sk.ERR_INVALID_ARG),
+    (9, {}, sk.ERR_UNSUPPORTED),
+    (2, dict(x=None), sk.ERR_INVALID_ARG),
+    (2, dict(w=None), sk.ERR_INVALID_ARG),
+    (2, dict(y=None), sk.ERR_INVALID_ARG),
+    (2, dict(N=0), sk.ERR_INVALID_ARG),
+    (2, dict(x=ALIGNED + 8), sk.ERR_ALIGNMENT),
+    (2, dict(w=ALIGNED + 4), sk.ERR_ALIGNMENT),
+    (2, dict(y=ALIGNED + 2), sk.ERR_ALIGNMENT),
+])
+def test_grouped_argument_checks(count, kw, status):
+    """Rejected before any CUDA call (the pointers are fake)."""
+    arr = _group(count, **kw)
+    st = sk.library().skinny_nvfp4_gemm_grouped(arr, count, 1, 512, sk.OUT_F32, None, 0, None)
+    assert st == status, sk.status_string(st)
+
+
+def test_grouped_rejects_bad_m_k_and_dtype():
+    arr = _group(2)
+    lib = sk.library()
+    assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 9, 512, sk.OUT_F32, None, 0, None) == sk.ERR_UNSUPPORTED
+    assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 520, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
+    assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 512, 3, None, 0, None) == sk.ERR_INVALID_ARG
+    assert lib.skinny_nvfp4_gemm_grouped(None, 2, 1, 512, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
