@@ -191,9 +191,18 @@ def build_device_workload(dev):
             for c in range(COPIES):
                 weights[c].append(sk.PackedFP8(pc if c == 0 else pc.clone(), s if c == 0 else s.clone(),
                                                spec.N, spec.K))
-    # Every activation and every output of a step lives in one contiguous
-    # device buffer (views per GEMM, 256-byte aligned), so that the end-to-end
-    # pass moves a step's inputs and results with one copy each way.
+    xs, ys = make_io_buffers(dev)
+    need = max(sk.workspace_bytes(w.fmt, M, w.N, w.K) for w in weights[0] for M in PASSES)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    return weights, xs, ys, ws
+
+
+def make_io_buffers(dev):
+    """Every activation and every output of a step in one contiguous device
+    buffer each (views per GEMM, 256-byte aligned), so that the end-to-end pass
+    moves a step's inputs and results with one copy each way."""
+    import torch
+
     xs, ys = {}, {}
     x_parts = [(M, i, si.activations(M, spec.K, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=100 + i))
                for M in PASSES for i, spec in enumerate(si.MIXED_LAYER)]
@@ -213,9 +222,7 @@ def build_device_workload(dev):
         ys.setdefault(M, []).append(y_buf[off:off + b].view(dt).view(M, spec.N))
         off += _padded(b)
     xs["buffer"], ys["buffer"] = x_buf, y_buf
-    need = max(sk.workspace_bytes(w.fmt, M, w.N, w.K) for w in weights[0] for M in PASSES)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
-    return weights, xs, ys, ws
+    return xs, ys
 
 
 def _padded(nbytes: int) -> int:
@@ -432,49 +439,75 @@ def launch_one(y, x, w, ws):
 
 
 def e2e_run(weights, xs, ys, ws, steps: int, warmup: int):
-    """Same workload through the public API with host buffers: every step copies
-    all its activations from pinned host memory (one copy: they share one
-    device buffer), runs the ten GEMMs, and reads all its outputs back (one
-    copy), in stream order."""
+    """Same workload through the public API with host buffers.  Every step
+    copies all its activations from pinned host memory to the device (one
+    copy: they share one device buffer), runs the ten GEMMs (one CUDA graph),
+    and reads all its outputs back to pinned host memory (one copy).  The
+    activations and outputs are double-buffered on the device: step i's
+    copy-in runs on one copy stream while step i-1's GEMMs run, and step i-1's
+    read-back on another, ordered by events (a buffer is refilled only after
+    the GEMMs two steps back have read it, and overwritten only after its
+    read-back).  Every step's copies are inside the timed region."""
     import torch
 
-    import fp8_weight_only_w4a16_b200 as sk
+    dev = xs["buffer"].device
+    bufs = [(xs, ys), make_io_buffers(dev)]
+    hx = xs["buffer"].cpu().pin_memory()
+    hys = [torch.empty(ys["buffer"].shape, dtype=ys["buffer"].dtype).pin_memory() for _ in range(2)]
+    h2d = xs["buffer"].numel()
+    d2h = ys["buffer"].numel()
 
-    x_buf, y_buf = xs["buffer"], ys["buffer"]
-    hx = x_buf.cpu().pin_memory()
-    hy = torch.empty(y_buf.shape, dtype=y_buf.dtype).pin_memory()
-    h2d = x_buf.numel()
-    d2h = y_buf.numel()
-
-    def one(step):
-        x_buf.copy_(hx, non_blocking=True)
-        for pi, M in enumerate(PASSES):
-            wc = weights[copy_for(step, pi)]
-            for i in range(len(si.MIXED_LAYER)):
-                sk.gemm_into(ys[M][i], xs[M][i], wc[i], workspace=ws)
-        hy.copy_(y_buf, non_blocking=True)
-
-    graphs = []
-    stream = torch.cuda.Stream()
-    stream.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(stream):
-        one(0)
-    torch.cuda.current_stream().wait_stream(stream)
+    graphs = {}
+    compute = torch.cuda.Stream()
+    compute.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(compute):
+        for b, (bx, by) in enumerate(bufs):
+            launch_step(weights, bx, by, ws, 0)
     torch.cuda.synchronize()
-    for phase in range(COPIES):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            one(phase)
-        graphs.append(g)
+    for b, (bx, by) in enumerate(bufs):
+        for phase in range(COPIES):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                launch_step(weights, bx, by, ws, phase)
+            graphs[phase, b] = g
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+    in_done = [ev(), ev()]
+    gemm_done = [ev(), ev()]
+    out_done = [ev(), ev()]
+    for b in range(2):   # every buffer starts free
+        gemm_done[b].record(compute)
+        out_done[b].record(s_out)
+
+    def one(i):
+        b = i % 2
+        x_buf, y_buf = bufs[b][0]["buffer"], bufs[b][1]["buffer"]
+        s_in.wait_event(gemm_done[b])            # the GEMMs of step i-2 have read x_buf
+        with torch.cuda.stream(s_in):
+            x_buf.copy_(hx, non_blocking=True)
+        in_done[b].record(s_in)
+        compute.wait_event(in_done[b])
+        compute.wait_event(out_done[b])          # step i-2's outputs have been read back
+        with torch.cuda.stream(compute):
+            graphs[i % COPIES, b].replay()
+        gemm_done[b].record(compute)
+        s_out.wait_event(gemm_done[b])
+        with torch.cuda.stream(s_out):
+            hys[b].copy_(y_buf, non_blocking=True)
+        out_done[b].record(s_out)
+
     for i in range(warmup):
-        graphs[i % COPIES].replay()
+        one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(compute)
+    s_in.wait_stream(compute)
     for i in range(steps):
-        graphs[i % COPIES].replay()
-    e1.record()
+        one(warmup + i)
+    compute.wait_stream(s_out)
+    e1.record(compute)
     torch.cuda.synchronize()
+    del graphs
     return e0.elapsed_time(e1), h2d, d2h
 
 

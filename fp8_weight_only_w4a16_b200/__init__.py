@@ -1,4 +1,4 @@
-"""B200-native weight-only skinny GEMM: y[M,N] = x[M,K] . W^T, M = 1..8,
+"""B200-native weight-only skinny GEMM: y[M,N] = x[M,K] . W^T, M = 1..16,
 with W kept in HBM as NVFP4 (E2M1 codes + UE4M3 per-16 scales + FP32 global)
 or FP8 E4M3 (+ FP32 per output channel), FP16 activations, FP32 accumulation.
 
@@ -31,7 +31,7 @@ OUT_F16 = 0
 OUT_F32 = 1
 FMT_NVFP4 = 0
 FMT_FP8 = 1
-MAX_M = 8
+MAX_M = 16
 MAX_GROUP = 8
 
 _lock = threading.Lock()

@@ -1,5 +1,5 @@
 // skinny.cu -- sm_100a kernels and C ABI of the weight-only skinny GEMM
-//   y[M,N] = x[M,K] . W^T,  M = 1..8,  W in NVFP4 (E2M1 + UE4M3/16 + FP32) or
+//   y[M,N] = x[M,K] . W^T,  M = 1..16, W in NVFP4 (E2M1 + UE4M3/16 + FP32) or
 //   FP8 E4M3 (+ FP32 per output channel), x FP16, FP32 accumulation.
 //
 // The operation is the decode-time weight-only GEMM of the v100-skinny pages
@@ -85,6 +85,12 @@ __device__ unsigned int g_device_error;
 // once, at the end of the kernel.
 __shared__ unsigned long long s_argmax_best[SKINNY_MAX_M];
 
+// Tokens are the n = 8 columns of the m16n8k16 MMA: a launch with M <= 8
+// runs one token block (NB = 1), one with 9 <= M <= 16 runs two (NB = 2),
+// each decoded weight fragment feeding NB MMAs.
+constexpr int kBlockTokens = 8;
+static_assert(SKINNY_MAX_M == 2 * kBlockTokens, "at most two token blocks");
+
 template <int FMT>
 struct Tile;
 
@@ -108,20 +114,22 @@ struct Tile<SKINNY_FMT_FP8> {
 };
 
 // Shared memory: kStages ring stages (one tile each), then the flush exchange
-// buffer (two parities of 16 warps x 2 strips x 32 lanes x float4), then the
-// mbarriers and the per-slot release counters, then (NVFP4) the buffer of the
-// fused SiLU*mul epilogue.
-template <int FMT>
+// buffer (two parities of 16 warps x 2 strips x NB token blocks x 32 lanes x
+// float4), then the mbarriers and the per-slot release counters, then (NVFP4)
+// the buffer of the fused SiLU*mul epilogue.  With two token blocks the FP8
+// ring has two slots (three do not fit next to the doubled exchange buffer).
+template <int FMT, int NB>
 struct Smem {
-    static constexpr int kStages = Tile<FMT>::kStages;
+    static constexpr int kStages = (FMT == SKINNY_FMT_FP8 && NB == 2) ? 2 : Tile<FMT>::kStages;
     static constexpr int kStageBytes = Tile<FMT>::kBytes;
     static constexpr int kXchgOff = kStages * kStageBytes;
-    static constexpr int kXchgBytes = 2 * kConsumerWarps * 2 * 32 * 16;
+    static constexpr int kXchgFloat4 = kConsumerWarps * 2 * NB * 32;   // one parity
+    static constexpr int kXchgBytes = 2 * kXchgFloat4 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
     static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
-    // Fused SiLU*mul epilogue (NVFP4 only): a finished row tile's outputs, [128 rows][8 tokens] FP32.
+    // Fused SiLU*mul epilogue (NVFP4 only): a finished row tile's outputs, [128 rows][8 NB tokens] FP32.
     static constexpr int kActOff = (kCountOff + kStages * 4 + 15) / 16 * 16;
-    static constexpr int kActBytes = FMT == SKINNY_FMT_NVFP4 ? kTileRows * SKINNY_MAX_M * 4 : 0;
+    static constexpr int kActBytes = FMT == SKINNY_FMT_NVFP4 ? kTileRows * kBlockTokens * NB * 4 : 0;
     static constexpr int kBytes = kActOff + kActBytes;
     static_assert(kStageBytes % 16 == 0, "stage alignment");
     // 227 KB per CTA; the static shared variables (fused argmax) take 128 B more.
@@ -146,7 +154,7 @@ struct Member {
 struct Params {
     Member mem[SKINNY_MAX_GROUP];
     int n_members;
-    uint2* partials;              // [P][16 warps][32 lanes] encoded float pairs (split-K only)
+    uint2* partials;              // [P][16 warps][32 lanes][NB] encoded float pairs (split-K only)
     int M, K;
     int C;                        // K tiles per row tile
     int U;                        // tiles in total (G * C)
@@ -242,9 +250,11 @@ __device__ __forceinline__ float argmax_key_value(unsigned long long key)
 __device__ __forceinline__ int argmax_key_row(unsigned long long key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
 // One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
-// tokens 2t and 2t+1 of this lane (v[0], v[1]).  Called by all 32 lanes.
+// tokens tok0 + 2t and tok0 + 2t + 1 of this lane (v[0], v[1]).  Called by
+// all 32 lanes.
 template <int FMT>
-__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane)
+__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
+                                         int tok0)
 {
     const int gid = lane >> 2, t = lane & 3;
     const Member& mb = p.mem[member_of(p, g)];
@@ -257,7 +267,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
         // The value is the one the FP32-output GEMM would store.
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int m = 2 * t + e;
+            const int m = tok0 + 2 * t + e;
             unsigned long long key = (n < mb.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
 #pragma unroll
             for (int d = 4; d < 32; d <<= 1) {
@@ -271,7 +281,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
     if (n >= mb.N) return;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-        const int m = 2 * t + e;
+        const int m = tok0 + 2 * t + e;
         if (m >= p.M) continue;
         const size_t idx = (size_t)m * mb.N + n;
         // Rounded FP32 product, never contracted with the add below, so the
@@ -294,42 +304,52 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
 // 0..63 of the tile are gate rows 64g.., rows 64..127 the matching up rows,
 // so the tile yields outputs j = 64g + 0..63 of every token:
 // y[m][j] = silu(gate) * up, silu(z) = z / (1 + e^-z), in FP32.
-template <int FMT>
-__device__ void silu_mul_epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
+template <int FMT, int NB>
+__device__ void silu_mul_epilogue(const Params& p, const float (&v)[NB][2], int g, int strip, int h, int lane,
                                   uint8_t* smem)
 {
-    float* act = reinterpret_cast<float*>(smem + Smem<FMT>::kActOff);   // [128 rows][8 tokens]
+    constexpr int kTok = kBlockTokens * NB;
+    float* act = reinterpret_cast<float*>(smem + Smem<FMT, NB>::kActOff);   // [128 rows][kTok tokens]
     const int gid = lane >> 2, t = lane & 3;
     const int r = strip * kStripRows + gid + 8 * h;
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
     const Member& mb = p.mem[0];   // the fused SiLU*mul runs one GEMM per launch
-    act[r * SKINNY_MAX_M + 2 * t] = v[0] * mb.out_scale;
-    act[r * SKINNY_MAX_M + 2 * t + 1] = v[1] * mb.out_scale;
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        act[r * kTok + kBlockTokens * nb + 2 * t] = v[nb][0] * mb.out_scale;
+        act[r * kTok + kBlockTokens * nb + 2 * t + 1] = v[nb][1] * mb.out_scale;
+    }
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    const int jl = threadIdx.x % 64, m = threadIdx.x / 64;          // 64 outputs x 8 tokens
+    const int jl = threadIdx.x % 64;                                  // 64 outputs x 8 tokens per pass
     const int F = mb.N / 2, j = g * 64 + jl;
-    if (m < p.M && j < F) {
-        const float gate = act[jl * SKINNY_MAX_M + m], up = act[(64 + jl) * SKINNY_MAX_M + m];
-        const float val = gate / (1.f + expf(-gate)) * up;
-        const size_t idx = (size_t)m * F + j;
-        if (p.out_f32)
-            static_cast<float*>(mb.y)[idx] = val;
-        else
-            static_cast<__half*>(mb.y)[idx] = __float2half_rn(val);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const int m = threadIdx.x / 64 + kBlockTokens * nb;
+        if (m < p.M && j < F) {
+            const float gate = act[jl * kTok + m], up = act[(64 + jl) * kTok + m];
+            const float val = gate / (1.f + expf(-gate)) * up;
+            const size_t idx = (size_t)m * F + j;
+            if (p.out_f32)
+                static_cast<float*>(mb.y)[idx] = val;
+            else
+                static_cast<__half*>(mb.y)[idx] = __float2half_rn(val);
+        }
     }
 }
 
 // The finished outputs of row tile g (this warp's slice) go to y, to the
 // fused argmax, or through the fused SiLU*mul.  Called by every warp of the
 // CTA together.
-template <int FMT>
-__device__ __forceinline__ void finish(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
+template <int FMT, int NB>
+__device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2], int g, int strip, int h, int lane,
                                        uint8_t* smem)
 {
-    if (FMT == SKINNY_FMT_NVFP4 && p.silu_mul)
-        silu_mul_epilogue<FMT>(p, v, g, strip, h, lane, smem);
-    else
-        epilogue<FMT>(p, v, g, strip, h, lane);
+    if (FMT == SKINNY_FMT_NVFP4 && p.silu_mul) {
+        silu_mul_epilogue<FMT, NB>(p, v, g, strip, h, lane, smem);
+    } else {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) epilogue<FMT>(p, v[nb], g, strip, h, lane, kBlockTokens * nb);
+    }
 }
 
 // Finish (or contribute to) row tile g, whose K range CTAs c_first..c_last
@@ -345,54 +365,72 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[2], int
 //    outputs, and zero the slots for the next call.
 // Which case applies is the same for every warp of the CTA, so the barriers
 // of the exchange and of the fused epilogues are reached by all of them.
-template <int FMT>
-__device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_first, int c_last, int parity,
+// With two token blocks every lane carries both blocks' sums (NB pairs).
+template <int FMT, int NB>
+__device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int c_first, int c_last, int parity,
                       uint8_t* smem, int b, int warp, int lane)
 {
-    float4* xchg = reinterpret_cast<float4*>(smem + Smem<FMT>::kXchgOff) + parity * (kConsumerWarps * 64);
+    using S = Smem<FMT, NB>;
+    float4* xchg = reinterpret_cast<float4*>(smem + S::kXchgOff) + parity * S::kXchgFloat4;
     const int sp = warp % kStripPairs, kq = warp / kStripPairs;
     const int sq = kq >> 1, h = kq & 1;          // this warp finishes strip 2sp+sq, rows gid+8h
-    xchg[warp * 64 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-    xchg[warp * 64 + 32 + lane] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    float tot[2] = {0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < kChunkPairs; ++k) {
-        const float4 v = xchg[(k * kStripPairs + sp) * 64 + sq * 32 + lane];
-        tot[0] += h ? v.z : v.x;
-        tot[1] += h ? v.w : v.y;
-    }
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+            xchg[((warp * 2 + q) * NB + nb) * 32 + lane] =
+                make_float4(acc[q][nb][0], acc[q][nb][1], acc[q][nb][2], acc[q][nb][3]);
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
+    float tot[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) tot[nb][0] = tot[nb][1] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kChunkPairs; ++k)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const float4 v = xchg[(((k * kStripPairs + sp) * 2 + sq) * NB + nb) * 32 + lane];
+            tot[nb][0] += h ? v.z : v.x;
+            tot[nb][1] += h ? v.w : v.y;
+        }
     const int strip = 2 * sp + sq;
     if (c_first == c_last) {
-        finish<FMT>(p, tot, g, strip, h, lane, smem);
+        finish<FMT, NB>(p, tot, g, strip, h, lane, smem);
         return;
     }
+    uint2* const mine = p.partials + ((b * kConsumerWarps + warp) * 32 + lane) * NB;
     if (b != c_last) {
-        ptx::st_volatile_v2(p.partials + (b * kConsumerWarps + warp) * 32 + lane,
-                            make_uint2(encode_partial(tot[0]), encode_partial(tot[1])));
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+            ptx::st_volatile_v2(mine + nb, make_uint2(encode_partial(tot[nb][0]), encode_partial(tot[nb][1])));
         return;
     }
     // Finisher.  The other contributors are lower-numbered CTAs; all but the
     // middle ones (whose whole range lies in g) published long ago.
-    constexpr int kBatch = 8;
-    float sum[2] = {0.f, 0.f};
+    constexpr int kBatch = 8 / NB;
+    float sum[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = 0.f;
     bool timed_out = false;
     uint64_t t0 = 0;
     for (int c0 = c_first; c0 < c_last; c0 += kBatch) {
-        uint2 v[kBatch];
+        uint2 v[kBatch][NB];
+        auto slot = [&](int k) { return p.partials + (((c0 + k) * kConsumerWarps + warp) * 32 + lane) * NB; };
 #pragma unroll
         for (int k = 0; k < kBatch; ++k)
-            v[k] = (c0 + k < c_last) ? ptx::ld_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane)
-                                     : make_uint2(1u, 1u);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                v[k][nb] = (c0 + k < c_last) ? ptx::ld_volatile_v2(slot(k) + nb) : make_uint2(1u, 1u);
         for (uint32_t it = 0;; ++it) {
             bool missing = false;
 #pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                if (v[k].x == 0u || v[k].y == 0u) {
-                    missing = true;
-                    v[k] = ptx::ld_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane);
+            for (int k = 0; k < kBatch; ++k)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    if (v[k][nb].x == 0u || v[k][nb].y == 0u) {
+                        missing = true;
+                        v[k][nb] = ptx::ld_volatile_v2(slot(k) + nb);
+                    }
                 }
-            }
             if (!missing || timed_out) break;
             if (it == 0) t0 = ptx::globaltimer_ns();
             else if ((it & 15u) == 0 && ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -403,28 +441,35 @@ __device__ void flush(const Params& p, const float (&acc)[2][4], int g, int c_fi
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
             if (c0 + k < c_last) {
-                sum[0] += decode_partial(v[k].x);
-                sum[1] += decode_partial(v[k].y);
-                ptx::st_volatile_v2(p.partials + ((c0 + k) * kConsumerWarps + warp) * 32 + lane, make_uint2(0u, 0u));
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    sum[nb][0] += decode_partial(v[k][nb].x);
+                    sum[nb][1] += decode_partial(v[k][nb].y);
+                    ptx::st_volatile_v2(slot(k) + nb, make_uint2(0u, 0u));
+                }
             }
         }
     }
-    sum[0] += tot[0];
-    sum[1] += tot[1];
-    finish<FMT>(p, sum, g, strip, h, lane, smem);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        sum[nb][0] += tot[nb][0];
+        sum[nb][1] += tot[nb][1];
+    }
+    finish<FMT, NB>(p, sum, g, strip, h, lane, smem);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.
-template <int FMT>
+template <int FMT, int NB>
 __device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int u)
 {
     const Member& mb = p.mem[member_of(p, u / p.C)];
     const uint8_t* src = mb.codes + (size_t)(u - mb.g_begin * p.C) * Tile<FMT>::kBytes;
     ptx::mbar_arrive_expect_tx(&full[s], Tile<FMT>::kBytes);
-    ptx::bulk_g2s(smem + s * Smem<FMT>::kStageBytes, src, Tile<FMT>::kBytes, &full[s], ptx::policy_evict_first());
+    ptx::bulk_g2s(smem + s * Smem<FMT, NB>::kStageBytes, src, Tile<FMT>::kBytes, &full[s],
+                  ptx::policy_evict_first());
 }
 
-// The B fragments of one K tile for this lane: token gid (row xrow of x),
+// The B fragments of one K tile for this lane: one token (row xrow of x),
 // logical columns [kb, kb+16), as 8 f16x2 words read straight from x
 // (read-only, L1-cached).  Tokens >= M (valid = false) and columns >= K read
 // as zero; K % 16 == 0, so the 16 columns are all in range or all out.
@@ -441,15 +486,15 @@ __device__ __forceinline__ void load_b(const uint16_t* xrow, bool valid, int kb,
 }
 
 // Per-warp state of the consumer loop.  A warp owns strips 2sp, 2sp+1 and K
-// chunks 2kq, 2kq+1 of every tile: four strip chunks, each with
-// its own accumulator chain (hiding the tensor-core latency); the two chunk
-// accumulators of a strip are added in a fixed order when a row tile is
+// chunks 2kq, 2kq+1 of every tile: four strip chunks, each with its own
+// accumulator chain per token block (hiding the tensor-core latency); the two
+// chunk accumulators of a strip are added in a fixed order when a row tile is
 // flushed.
-template <int FMT>
+template <int FMT, int NB>
 struct Consumer {
-    float acc[2][2][4];     // [chunk parity][strip][fragment]
-    uint32_t lane_codes;    // this lane's code bytes of strip 2sp, chunk 2kq, inside a tile
-    uint32_t lane_scale;    // this lane's scale word of strip 2sp, chunk 2kq (NVFP4)
+    float acc[2][2][NB][4];   // [chunk parity][strip][token block][fragment]
+    uint32_t lane_codes;      // this lane's code bytes of strip 2sp, chunk 2kq, inside a tile
+    uint32_t lane_scale;      // this lane's scale word of strip 2sp, chunk 2kq (NVFP4)
 
     __device__ __forceinline__ void zero()
     {
@@ -458,23 +503,27 @@ struct Consumer {
 #pragma unroll
             for (int q = 0; q < 2; ++q)
 #pragma unroll
-                for (int r = 0; r < 4; ++r) acc[u][q][r] = 0.f;
+                for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[u][q][nb][r] = 0.f;
     }
 
     // The per-strip sums of both chunks (fixed order).
-    __device__ __forceinline__ void total(float (&tot)[2][4]) const
+    __device__ __forceinline__ void total(float (&tot)[2][NB][4]) const
     {
 #pragma unroll
         for (int q = 0; q < 2; ++q)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) tot[q][r] = acc[0][q][r] + acc[1][q][r];
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) tot[q][nb][r] = acc[0][q][nb][r] + acc[1][q][nb][r];
     }
 
     // The warp's four strip chunks of the tile at shared address `tile`;
-    // bx[u] holds the activations of chunk 2kq + u.  All shared loads are
-    // issued first, then the decode and MMA steps of the four chains
-    // interleave.
-    __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][8])
+    // bx[u][nb] holds the activations of chunk 2kq + u for token block nb.
+    // All shared loads are issued first, then the decode and MMA steps of the
+    // chains interleave; each decoded fragment feeds one MMA per token block.
+    __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][NB][8])
     {
         if constexpr (FMT == SKINNY_FMT_NVFP4) {
             uint4 cw[2][2];
@@ -504,7 +553,9 @@ struct Consumer {
                         ptx::e2m1x8_to_f16x8(w, h);
                         const uint32_t a[4] = {ptx::hmul2(h[0], s0[u][q]), ptx::hmul2(h[1], s8[u][q]),
                                                ptx::hmul2(h[2], s0[u][q]), ptx::hmul2(h[3], s8[u][q])};
-                        ptx::mma_f16_16816(acc[u][q], a, bx[u][2 * j], bx[u][2 * j + 1]);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+                            ptx::mma_f16_16816(acc[u][q][nb], a, bx[u][nb][2 * j], bx[u][nb][2 * j + 1]);
                     }
         } else {
             uint4 cw[2][2][2];
@@ -527,23 +578,30 @@ struct Consumer {
                         uint32_t a[4];
                         ptx::e4m3x4_to_f16x4(w0, a[0], a[1]);
                         ptx::e4m3x4_to_f16x4(w1, a[2], a[3]);
-                        ptx::mma_f16_16816(acc[u][q], a, bx[u][2 * j], bx[u][2 * j + 1]);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+                            ptx::mma_f16_16816(acc[u][q][nb], a, bx[u][nb][2 * j], bx[u][nb][2 * j + 1]);
                     }
         }
     }
 };
 
-template <int FMT>
+// The consumer loop of one warp over the CTA's range of tiles.  With one
+// token block the activations of the next tile are fetched one tile ahead
+// into ping-pong registers; with two there is no room for a second set, and
+// each tile's activations are fetched as the tile begins (before its wait).
+template <int FMT, int NB>
 __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, const Sched& sc, int warp,
                         int lane)
 {
-    using S = Smem<FMT>;
+    using S = Smem<FMT, NB>;
     constexpr int kStages = S::kStages;
+    constexpr bool kAhead = NB == 1;
     const int gid = lane >> 2, t = lane & 3;
     const int sp = warp % kStripPairs, kq = warp / kStripPairs;
     const int n_units = sc.n_units;
 
-    Consumer<FMT> w;
+    Consumer<FMT, NB> w;
     w.zero();
     if constexpr (FMT == SKINNY_FMT_NVFP4) {
         w.lane_codes = (2 * sp) * kNvfp4StripCodeBytes + (2 * kq) * 512 + lane * 16;
@@ -552,10 +610,15 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 16;
         w.lane_scale = 0;
     }
-    // Activations: token gid, columns c*512 + (2kq + u)*64 + [16t, 16t+16),
+    // Activations: tokens gid + 8nb, columns c*512 + (2kq + u)*64 + [16t, 16t+16),
     // from the x of the GEMM that owns the tile.
-    const bool xvalid = gid < p.M;
-    const size_t xoff = (size_t)(xvalid ? gid : 0) * p.K;
+    bool xvalid[NB];
+    size_t xoff[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        xvalid[nb] = gid + kBlockTokens * nb < p.M;
+        xoff[nb] = (size_t)(xvalid[nb] ? gid + kBlockTokens * nb : 0) * p.K;
+    }
     const int kb_lane = 2 * kq * kChunkK + 16 * t;
 
     // The range is walked from its last tile down to its first.
@@ -564,38 +627,39 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     int nc = c;                                            // K tile whose activations are fetched next
     int ng = g;                                            // ... and its row tile
     int nm = member_of(p, ng);                             // ... and its GEMM
-    const uint16_t* xrow = p.mem[nm].x + xoff;
+    const uint16_t* xbase = p.mem[nm].x;
     const uint32_t smem32 = ptx::smem_addr(smem);
     int* released = reinterpret_cast<int*>(smem + S::kCountOff);
     // Contributors of a row tile: only the two at the ends of the range are shared.
     auto flush_g = [&](int fg) {
-        float tot[2][4];
+        float tot[2][NB][4];
         w.total(tot);
         const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
         const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
-        flush<FMT>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane);
+        flush<FMT, NB>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane);
         parity ^= 1;
     };
-
-    uint32_t bx[2][2][8];   // ping-pong: [buffer][chunk][words]
-    load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, bx[0][0]);
-    load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, bx[0][1]);
+    auto fetch = [&](uint32_t (&dst)[2][NB][8]) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                load_b(xbase + xoff[nb], xvalid[nb], nc * kTileK + kb_lane + u * kChunkK, p.K, dst[u][nb]);
+    };
+    auto advance = [&]() {   // the fetch cursor moves one tile down the range
+        if (nc == 0) {
+            nc = p.C;
+            if (--ng < p.mem[nm].g_begin && nm > 0) xbase = p.mem[--nm].x;
+        }
+        --nc;
+    };
 
     bool ok = true;
     int s = 0;
     uint32_t phase = 0;
-    // One tile per iteration; the body is written for buffer B = i & 1 (the
-    // loop is unrolled by two so the ping-pong buffers stay in registers).
-    auto step = [&](int i, uint32_t (&cur)[2][8], uint32_t (&nxt)[2][8]) {
-        if (nc == 0) {
-            nc = p.C;
-            if (--ng < p.mem[nm].g_begin && nm > 0) xrow = p.mem[--nm].x + xoff;
-        }
-        --nc;
-        if (i + 1 < n_units) {   // next tile's activations, one tile ahead
-            load_b(xrow, xvalid, nc * kTileK + kb_lane, p.K, nxt[0]);
-            load_b(xrow, xvalid, nc * kTileK + kb_lane + kChunkK, p.K, nxt[1]);
-        }
+    // One tile: wait for its slot, flush the previous row tile if this one
+    // starts a new one, decode and multiply, release the slot.
+    auto body = [&](int i, const uint32_t (&cur)[2][NB][8]) {
         if (ok) {
             // All lanes agree on the outcome, so the warp stays converged.
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[s], phase, kWaitLimitNs));
@@ -616,7 +680,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
                     released[s] = 0;
                     if (i + kStages < n_units) {
                         if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
-                            issue_stage<FMT>(p, smem, full, s, sc.u_last - (i + kStages));
+                            issue_stage<FMT, NB>(p, smem, full, s, sc.u_last - (i + kStages));
                         else
                             atomicOr(&g_device_error, kErrEmptyWait);
                     }
@@ -633,12 +697,30 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         }
         --c;
     };
-    int i = 0;
-    for (; i + 1 < n_units; i += 2) {
-        step(i, bx[0], bx[1]);
-        step(i + 1, bx[1], bx[0]);
+
+    if constexpr (kAhead) {
+        uint32_t bx[2][2][NB][8];   // ping-pong: [buffer][chunk][token block][words]
+        fetch(bx[0]);
+        // The loop is unrolled by two so the ping-pong buffers stay in registers.
+        auto step = [&](int i, uint32_t (&cur)[2][NB][8], uint32_t (&nxt)[2][NB][8]) {
+            advance();
+            if (i + 1 < n_units) fetch(nxt);   // next tile's activations, one tile ahead
+            body(i, cur);
+        };
+        int i = 0;
+        for (; i + 1 < n_units; i += 2) {
+            step(i, bx[0], bx[1]);
+            step(i + 1, bx[1], bx[0]);
+        }
+        if (i < n_units) step(i, bx[0], bx[1]);
+    } else {
+        uint32_t bx[2][NB][8];
+        for (int i = 0; i < n_units; ++i) {
+            fetch(bx);
+            advance();
+            body(i, bx);
+        }
     }
-    if (i < n_units) step(i, bx[0], bx[1]);
 
     if (n_units > 0) flush_g(cur_g);
     if (!ok && threadIdx.x == 0) {
@@ -650,10 +732,10 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
 }
 
-template <int FMT>
+template <int FMT, int NB>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p)
 {
-    using S = Smem<FMT>;
+    using S = Smem<FMT, NB>;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
     uint64_t* empty = full + S::kStages;
@@ -672,14 +754,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         ptx::fence_mbar_init();
         // The packed weights are read-only parameters: start streaming them
         // before the previous kernel in the stream has finished.
-        for (int q = 0; q < S::kStages && q < sc.n_units; ++q) issue_stage<FMT>(p, smem, full, q, sc.u_last - q);
+        for (int q = 0; q < S::kStages && q < sc.n_units; ++q)
+            issue_stage<FMT, NB>(p, smem, full, q, sc.u_last - q);
     }
     __syncthreads();
     // x, y, the channel scales and the workspace may belong to the previous
     // kernel: touch them only once it has completed.
     ptx::pdl_wait_prior_grid();
 
-    consume<FMT>(p, smem, full, empty, sc, warp, lane);
+    consume<FMT, NB>(p, smem, full, empty, sc, warp, lane);
 
     if (p.argmax) {
         // The CTA that finishes last turns the maxima into (row, value) per
@@ -725,11 +808,14 @@ static int current_device(int* sms)
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             return SKINNY_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_NVFP4>::kBytes) != cudaSuccess)
-            return SKINNY_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_FP8>::kBytes) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_NVFP4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem<SKINNY_FMT_NVFP4, 1>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_NVFP4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem<SKINNY_FMT_NVFP4, 2>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_FP8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem<SKINNY_FMT_FP8, 1>::kBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_FP8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem<SKINNY_FMT_FP8, 2>::kBytes) != cudaSuccess)
             return SKINNY_ERR_CUDA;
         d.sms = n;
         d.ready = true;
@@ -738,10 +824,11 @@ static int current_device(int* sms)
     return SKINNY_OK;
 }
 
-// Workspace layout (identical for every shape on a device, so one workspace
-// can serve calls of different shapes in turn): one partial-sum slot of
-// 16 warps x 32 lanes x 2 floats per CTA, for up to one CTA per SM, then the
-// fused argmax's running maxima (one 64-bit key per token) and CTA counter.
+// Workspace layout (identical for every shape and M on a device, so one
+// workspace can serve calls of different shapes in turn): one partial-sum slot
+// of 16 warps x 32 lanes x 2 token blocks x 2 floats (8 KB) per CTA, for up to
+// one CTA per SM, then the fused argmax's running maxima (one 64-bit key per
+// token) and CTA counter.
 constexpr size_t kArgmaxTailBytes = 256;
 struct Plan {
     int G, C, U, P;
@@ -760,7 +847,7 @@ static int make_plan(int64_t G, int64_t K, int sms, bool split, Plan* pl)
     pl->U = (int)(G * C);
     const int UQ = split ? pl->U : pl->G;
     pl->P = UQ < sms ? UQ : sms;
-    pl->partial_bytes = (size_t)sms * kConsumerWarps * 32 * sizeof(uint2);
+    pl->partial_bytes = (size_t)sms * kConsumerWarps * 32 * 2 * sizeof(uint2);
     pl->workspace_bytes = pl->partial_bytes + kArgmaxTailBytes;
     return SKINNY_OK;
 }
@@ -824,17 +911,19 @@ static int launch(Params p, int64_t G, int64_t K, void* workspace, size_t worksp
     }
     // Programmatic dependent launch: the kernel may start (and prefetch its
     // weights) while the previous kernel in the stream is finishing.
+    const bool two_blocks = p.M > kBlockTokens;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.P);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = Smem<FMT>::kBytes;
+    cfg.dynamicSmemBytes = two_blocks ? Smem<FMT, 2>::kBytes : Smem<FMT, 1>::kBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<FMT>, p) != cudaSuccess) return SKINNY_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2> : gemm_kernel<FMT, 1>, p) != cudaSuccess)
+        return SKINNY_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SKINNY_OK : SKINNY_ERR_CUDA;
 }
 

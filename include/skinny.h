@@ -1,7 +1,7 @@
 /*
  * skinny.h -- C ABI of the B200 weight-only skinny GEMM library (libskinny.so).
  *
- *   y[M,N] = x[M,K] . W^T,   M = 1..8 rows, W kept compressed in HBM.
+ *   y[M,N] = x[M,K] . W^T,   M = 1..16 rows, W kept compressed in HBM.
  *
  * The operation.  During single-request decode (one token, or a k=7
  * speculative-verify round plus its base token: 8 rows), a language model's
@@ -58,7 +58,7 @@ extern "C" {
 typedef enum {
     SKINNY_OK = 0,
     SKINNY_ERR_INVALID_ARG = -1,  /* null pointer, K % 16 != 0, N or K <= 0, bad dtype, bad scale byte */
-    SKINNY_ERR_UNSUPPORTED = -2,  /* M outside [1, 8], or a size past the library's limits */
+    SKINNY_ERR_UNSUPPORTED = -2,  /* M outside [1, 16], or a size past the library's limits */
     SKINNY_ERR_ALIGNMENT = -3,    /* a device pointer is not aligned as documented */
     SKINNY_ERR_CUDA = -4,         /* a CUDA runtime call failed (launch, attribute, device query) */
     SKINNY_ERR_WORKSPACE = -5     /* workspace non-null but smaller than skinny_workspace_bytes() */
@@ -68,7 +68,7 @@ typedef enum { SKINNY_OUT_F16 = 0, SKINNY_OUT_F32 = 1 } skinny_out_dtype;
 
 typedef enum { SKINNY_FMT_NVFP4 = 0, SKINNY_FMT_FP8 = 1 } skinny_format;
 
-#define SKINNY_MAX_M 8
+#define SKINNY_MAX_M 16
 
 /* Most GEMMs one skinny_nvfp4_gemm_grouped call can run. */
 #define SKINNY_MAX_GROUP 8
@@ -128,7 +128,7 @@ int skinny_unpack_fp8(const void* w_packed, int64_t N, int64_t K, uint8_t* q);
  * ---------------------------------------------------------------------- */
 
 /* Size of the optional split-K workspace for one GEMM of this format and
- * shape on the CURRENT device (it depends on the SM count only: 4 KB per SM
+ * shape on the CURRENT device (it depends on the SM count only: 8 KB per SM
  * plus 256 bytes for the fused argmax's running maxima).
  * A workspace lets the kernel split K across CTAs so that every SM streams
  * the same number of weight bytes (a short-N shape such as 5120 x 5120 has
@@ -158,7 +158,9 @@ int skinny_workspace_bytes(int fmt, int M, int64_t N, int64_t K, size_t* bytes);
  * token and M=8 the k=7 verify round; aiwitness.kr post, section
  * "내가 실제로 만든 것").
  *   x            device [M][K] FP16, 16-byte aligned, read-only during the call.
- *   M            1..8 (rows of x: tokens of one decode / verify round).
+ *   M            1..16 (rows of x: the tokens of one decode step or verify
+ *                round: 1, or a base token plus k drafts; 9..16 covers a
+ *                deeper draft or two requests' verify rounds).
  *   K            multiple of 16.
  *   w_packed     device, from skinny_pack_nvfp4 (codes and block scales), 16-byte aligned.
  *   global_scale FP32 per-tensor scale, applied to the FP32 sum.
@@ -293,7 +295,7 @@ int skinny_nvfp4_gemm_grouped(const skinny_nvfp4_group_member* members, int coun
  * scratch lives in one static device array of skinny_static_workspace_capacity()
  * bytes (4 MiB) that every GPU which loads this library holds until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
- * allocating library routine.  The scratch needed is 4 KB per SM, whatever
+ * allocating library routine.  The scratch needed is 8 KB per SM, whatever
  * the shape; a device with more SMs than the array has slots for returns
  * SKINNY_ERR_UNSUPPORTED.
  *

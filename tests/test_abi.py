@@ -45,7 +45,7 @@ ALIGNED = 1 << 20  # a fake, 16-byte aligned address: never dereferenced by thes
     (dict(y=None), sk.ERR_INVALID_ARG),
     (dict(w=None), sk.ERR_INVALID_ARG),
     (dict(M=0), sk.ERR_UNSUPPORTED),
-    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(M=17), sk.ERR_UNSUPPORTED),
     (dict(K=24), sk.ERR_INVALID_ARG),
     (dict(K=0), sk.ERR_INVALID_ARG),
     (dict(N=0), sk.ERR_INVALID_ARG),
@@ -65,7 +65,7 @@ def test_nvfp4_argument_checks(kw, status):
 @pytest.mark.parametrize("kw,status", [
     (dict(scale=None), sk.ERR_INVALID_ARG),
     (dict(scale=ALIGNED + 2), sk.ERR_ALIGNMENT),
-    (dict(M=12), sk.ERR_UNSUPPORTED),
+    (dict(M=17), sk.ERR_UNSUPPORTED),
 ])
 def test_fp8_argument_checks(kw, status):
     a = dict(x=ALIGNED, M=2, K=64, w=ALIGNED, scale=ALIGNED, N=32, y=ALIGNED)
@@ -79,7 +79,7 @@ def test_workspace_query_argument_checks():
     lib = sk.library()
     assert lib.skinny_workspace_bytes(5, 1, 64, 64, ctypes.byref(b)) == sk.ERR_INVALID_ARG
     assert lib.skinny_workspace_bytes(0, 1, 64, 40, ctypes.byref(b)) == sk.ERR_INVALID_ARG
-    assert lib.skinny_workspace_bytes(0, 9, 64, 64, ctypes.byref(b)) == sk.ERR_UNSUPPORTED
+    assert lib.skinny_workspace_bytes(0, 17, 64, 64, ctypes.byref(b)) == sk.ERR_UNSUPPORTED
     assert lib.skinny_workspace_bytes(0, 1, 64, 64, None) == sk.ERR_INVALID_ARG
 
 
@@ -87,7 +87,7 @@ def test_workspace_query_argument_checks():
     (dict(idx=None), sk.ERR_INVALID_ARG),
     (dict(val=None), sk.ERR_INVALID_ARG),
     (dict(w=None), sk.ERR_INVALID_ARG),
-    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(M=17), sk.ERR_UNSUPPORTED),
     (dict(K=40), sk.ERR_INVALID_ARG),
     (dict(idx=ALIGNED + 2), sk.ERR_ALIGNMENT),
     (dict(val=ALIGNED + 2), sk.ERR_ALIGNMENT),
@@ -106,7 +106,7 @@ def test_nvfp4_argmax_argument_checks(kw, status):
     (dict(F=0), sk.ERR_INVALID_ARG),
     (dict(y=None), sk.ERR_INVALID_ARG),
     (dict(w=None), sk.ERR_INVALID_ARG),
-    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(M=17), sk.ERR_UNSUPPORTED),
     (dict(out=5), sk.ERR_INVALID_ARG),
     (dict(w=ALIGNED + 4), sk.ERR_ALIGNMENT),
 ])
@@ -123,7 +123,7 @@ def test_nvfp4_silu_mul_argument_checks(kw, status):
     (dict(res=None), sk.ERR_INVALID_ARG),
     (dict(res=ALIGNED + 2), sk.ERR_ALIGNMENT),
     (dict(y=None), sk.ERR_INVALID_ARG),
-    (dict(M=9), sk.ERR_UNSUPPORTED),
+    (dict(M=17), sk.ERR_UNSUPPORTED),
 ])
 def test_gemm_add_argument_checks(fmt, kw, status):
     a = dict(x=ALIGNED, M=2, K=64, w=ALIGNED, N=32, res=ALIGNED, y=ALIGNED)
@@ -206,7 +206,7 @@ def test_grouped_argument_checks(count, kw, status):
 def test_grouped_rejects_bad_m_k_and_dtype():
     arr = _group(2)
     lib = sk.library()
-    assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 9, 512, sk.OUT_F32, None, 0, None) == sk.ERR_UNSUPPORTED
+    assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 17, 512, sk.OUT_F32, None, 0, None) == sk.ERR_UNSUPPORTED
     assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 520, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
     assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 512, 3, None, 0, None) == sk.ERR_INVALID_ARG
     assert lib.skinny_nvfp4_gemm_grouped(None, 2, 1, 512, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
