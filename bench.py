@@ -329,6 +329,57 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, tri
     return out, best
 
 
+def grouped_attention_us(weights, xs, ys, ws, peak, launches: int = 30, replays: int = 3, trials: int = 10):
+    """The step's three 5120 x 5120 NVFP4 projections (q, kv, o: own x, own y)
+    as ONE grouped launch, at M = 1 and 8: per-launch device time (median and
+    best of `trials`), timed like the standalone GEMMs (graphs of back-to-back
+    launches over weight copies > 4x L2)."""
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    idx = [i for i, s in enumerate(si.MIXED_LAYER) if s.fmt == "nvfp4" and s.N == 5120 and s.K == 5120]
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    per_set = sum(weight_bytes(si.MIXED_LAYER[i]) for i in idx)
+    n_set = max(COPIES, int(np.ceil(4 * l2 / per_set)))
+    sets = [[weights[c][i] for i in idx] for c in range(COPIES)]
+    sets += [[clone_weight(weights[0][i]) for i in idx] for _ in range(n_set - COPIES)]
+    rows = []
+    stream = torch.cuda.Stream()
+    for M in PASSES:
+        xg = [xs[M][i] for i in idx]
+        yg = [ys[M][i] for i in idx]
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            sk.gemm_grouped_into(yg, xg, sets[0], workspace=ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(launches):
+                sk.gemm_grouped_into(yg, xg, sets[r % n_set], workspace=ws)
+        g.replay()
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(trials):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(replays):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t.append(1e3 * e0.elapsed_time(e1) / (replays * launches))
+        del g
+        b = sum(gemm_bytes(si.MIXED_LAYER[i], M) for i in idx)
+        us = float(np.median(t))
+        rows.append({"M": M, "us": round(us, 3), "us_best": round(float(np.min(t)), 3), "GB/s": round(b / us / 1e3, 1),
+                     "frac": round(b / us / 1e3 / peak, 4)})
+    del sets
+    torch.cuda.empty_cache()
+    return {"gemms": ["%s nvfp4 5120x5120" % si.MIXED_LAYER[i].name for i in idx], "passes": rows,
+            "note": "one skinny_nvfp4_gemm_grouped launch of the three attention projections; the step itself "
+                    "runs them as three launches"}
+
+
 def _random_packed_copies(dev, N, K, gen):
     """Packed NVFP4 tiles drawn on the device (random E2M1 codes, UE4M3 block
     scales in [2^-4, 2^4]), as many copies as it takes to exceed 4x L2."""
@@ -430,6 +481,51 @@ def fused_epilogues_us(dev, launches: int = 20, replays: int = 3):
         del copies, plain, gu, ws
         torch.cuda.empty_cache()
     return result
+
+
+READ_CEILING_BYTES = 4 << 30
+
+
+def read_only_ceiling(dev, trials: int = 5):
+    """The in-run read-only HBM ceiling: the library's streaming-read kernels
+    (16-byte loads from every thread, and 36 KB bulk copies into a shared-memory
+    ring) over a 4 GiB buffer, best of `trials` each, CUDA events on the
+    launching stream.  The faster method is the ceiling."""
+    import ctypes
+
+    import torch
+
+    import fp8_weight_only_w4a16_b200 as sk
+
+    buf = torch.empty(READ_CEILING_BYTES, dtype=torch.uint8, device=dev)
+    buf.random_(0, 256)   # the 16-byte loads could otherwise be fed by compressed zero pages
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    lib = sk.library()
+    stream = torch.cuda.current_stream()
+    out = {}
+    for method, name, nbytes in ((0, "ldg", READ_CEILING_BYTES),
+                                 (1, "bulk", READ_CEILING_BYTES // 36864 * 36864)):
+        def run():
+            st = lib.skinny_stream_read(ctypes.c_void_p(buf.data_ptr()), READ_CEILING_BYTES, method,
+                                        ctypes.c_void_p(sink.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+            if st != sk.OK:
+                raise sk.SkinnyError(st, "skinny_stream_read")
+        run()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(trials):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        out[name] = {"GB/s": round(nbytes / min(ts) / 1e9, 1), "GB/s_median": round(nbytes / float(np.median(ts)) / 1e9, 1),
+                     "bytes": nbytes}
+    del buf
+    torch.cuda.empty_cache()
+    best = max(v["GB/s"] for v in out.values())
+    return best, out
 
 
 def launch_one(y, x, w, ws):
@@ -689,6 +785,8 @@ def main(argv=None):
     # Per-launch device time of each GEMM (CUDA events around graphs of
     # back-to-back launches); this also brings the GPU to its loaded clocks.
     dur_us, best_us = per_launch_us(weights, xs, ys, ws)
+    ro_peak, ro_methods = read_only_ceiling(dev)
+    grouped = grouped_attention_us(weights, xs, ys, ws, peak)
     fused = fused_epilogues_us(dev)
 
     for i in range(args.warmup):
@@ -741,6 +839,9 @@ def main(argv=None):
         "frac_of_peak": round(value / world / peak, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_src,
+                     "peak_read_only": ro_peak, "frac_read_only": round(achieved / ro_peak, 4),
+                     "read_only_ceiling": dict(ro_methods, note="measured in this run: the library's read-only "
+                                               "streaming kernels over 4 GiB, best of 5; the faster is peak_read_only"),
                      "kernel": "gemm_kernel<NVFP4>", "launches_in_step": nv_launches,
                      "method": "per-launch device time from CUDA events around graphs of 30 back-to-back launches "
                                "of each GEMM over rotating weight copies > 4x L2, measured in this process before "
@@ -748,6 +849,7 @@ def main(argv=None):
                                "launches"},
         "sum_launch_us": round(float(dur_us.sum()), 2),
         "per_gemm": per,
+        "grouped_attention": grouped,
         "fused_epilogues": dict(fused, note="next rows: the per-token argmax, the SiLU*mul activation and the "
                                             "residual add fused into the GEMM epilogue, each next to the plain "
                                             "GEMM it replaces; per-launch device time, not part of the step"),

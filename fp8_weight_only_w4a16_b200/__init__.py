@@ -87,6 +87,7 @@ def library() -> ctypes.CDLL:
                 "skinny_nvfp4_gemm_silu_mul": (ctypes.c_int, [p, ctypes.c_int, i64, p, ctypes.c_float, i64, p,
                                                               ctypes.c_int, p, sz, p]),
                 "skinny_static_workspace_capacity": (sz, []),
+                "skinny_stream_read": (ctypes.c_int, [p, sz, ctypes.c_int, p, p]),
                 "skinny_nvfp4_gemm_grouped": (ctypes.c_int, [ctypes.POINTER(GroupMember), ctypes.c_int,
                                                              ctypes.c_int, i64, ctypes.c_int, p, sz, p]),
                 "skinny_debug_static_workspace_address": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p)]),

@@ -12,7 +12,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, "skinny.cu"), os.path.join(CSRC, "pack.cpp")]
+SOURCES = [os.path.join(CSRC, "skinny.cu"), os.path.join(CSRC, "stream_read.cu"), os.path.join(CSRC, "pack.cpp")]
 HEADERS = [os.path.join(CSRC, "layout.h"), os.path.join(CSRC, "ptx.cuh"), os.path.join(ROOT, "include", "skinny.h")]
 LIBRARY = os.path.join(PKG, "libskinny.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -250,11 +250,12 @@ __device__ __forceinline__ float argmax_key_value(unsigned long long key)
 __device__ __forceinline__ int argmax_key_row(unsigned long long key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
 // One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
-// tokens tok0 + 2t and tok0 + 2t + 1 of this lane (v[0], v[1]).  Called by
+// tokens tok0 + 2t and tok0 + 2t + 1 of this lane (v[0], v[1]; res[0],
+// res[1] the residual of those outputs when the GEMM adds one).  Called by
 // all 32 lanes.
 template <int FMT>
-__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], int g, int strip, int h, int lane,
-                                         int tok0)
+__device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], const float (&res)[2], int g,
+                                         int strip, int h, int lane, int tok0)
 {
     const int gid = lane >> 2, t = lane & 3;
     const Member& mb = p.mem[member_of(p, g)];
@@ -288,11 +289,9 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], i
         // fused add sees exactly the value the plain GEMM stores.
         float val = __fmul_rn(v[e], sc);
         // Fused residual add: one FP32 add, then the single output rounding.
-        // Each element is read and written by this thread only, so the
-        // residual may be y itself.
-        if (mb.residual)
-            val = __fadd_rn(val, p.out_f32 ? static_cast<const float*>(mb.residual)[idx]
-                                           : __half2float(static_cast<const __half*>(mb.residual)[idx]));
+        // Each element is read (early, by load_residual) and written by this
+        // thread only, so the residual may be y itself.
+        if (mb.residual) val = __fadd_rn(val, res[e]);
         if (p.out_f32)
             static_cast<float*>(mb.y)[idx] = val;
         else
@@ -337,18 +336,43 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[NB][2], int 
     }
 }
 
+// The residual of this lane's outputs of row tile g (strip `strip`, rows
+// gid + 8h, tokens 8nb + 2t + e), loaded as soon as the CTA knows that it
+// finishes the row tile, so that the loads overlap the exchange and the
+// split-K wait instead of stalling the epilogue.  Zero where there is none.
+template <int NB>
+__device__ __forceinline__ void load_residual(const Params& p, int g, int strip, int h, int lane,
+                                              float (&res)[NB][2])
+{
+    const int gid = lane >> 2, t = lane & 3;
+    const Member& mb = p.mem[member_of(p, g)];
+    const int n = (g - mb.g_begin) * kTileRows + strip * kStripRows + gid + 8 * h;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int m = kBlockTokens * nb + 2 * t + e;
+            res[nb][e] = 0.f;
+            if (mb.residual && n < mb.N && m < p.M) {
+                const size_t idx = (size_t)m * mb.N + n;
+                res[nb][e] = p.out_f32 ? static_cast<const float*>(mb.residual)[idx]
+                                       : __half2float(static_cast<const __half*>(mb.residual)[idx]);
+            }
+        }
+}
+
 // The finished outputs of row tile g (this warp's slice) go to y, to the
 // fused argmax, or through the fused SiLU*mul.  Called by every warp of the
 // CTA together.
 template <int FMT, int NB>
-__device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2], int g, int strip, int h, int lane,
-                                       uint8_t* smem)
+__device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2], const float (&res)[NB][2], int g,
+                                       int strip, int h, int lane, uint8_t* smem)
 {
     if (FMT == SKINNY_FMT_NVFP4 && p.silu_mul) {
         silu_mul_epilogue<FMT, NB>(p, v, g, strip, h, lane, smem);
     } else {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) epilogue<FMT>(p, v[nb], g, strip, h, lane, kBlockTokens * nb);
+        for (int nb = 0; nb < NB; ++nb) epilogue<FMT>(p, v[nb], res[nb], g, strip, h, lane, kBlockTokens * nb);
     }
 }
 
@@ -374,6 +398,9 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
     float4* xchg = reinterpret_cast<float4*>(smem + S::kXchgOff) + parity * S::kXchgFloat4;
     const int sp = warp % kStripPairs, kq = warp / kStripPairs;
     const int sq = kq >> 1, h = kq & 1;          // this warp finishes strip 2sp+sq, rows gid+8h
+    const int strip = 2 * sp + sq;
+    float res[NB][2];
+    if (c_first == c_last || b == c_last) load_residual<NB>(p, g, strip, h, lane, res);
 #pragma unroll
     for (int q = 0; q < 2; ++q)
 #pragma unroll
@@ -392,9 +419,8 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
             tot[nb][0] += h ? v.z : v.x;
             tot[nb][1] += h ? v.w : v.y;
         }
-    const int strip = 2 * sp + sq;
     if (c_first == c_last) {
-        finish<FMT, NB>(p, tot, g, strip, h, lane, smem);
+        finish<FMT, NB>(p, tot, res, g, strip, h, lane, smem);
         return;
     }
     uint2* const mine = p.partials + ((b * kConsumerWarps + warp) * 32 + lane) * NB;
@@ -455,7 +481,7 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
         sum[nb][0] += tot[nb][0];
         sum[nb][1] += tot[nb][1];
     }
-    finish<FMT, NB>(p, sum, g, strip, h, lane, smem);
+    finish<FMT, NB>(p, sum, res, g, strip, h, lane, smem);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.

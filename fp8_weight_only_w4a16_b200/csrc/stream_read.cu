@@ -1,0 +1,115 @@
+// stream_read.cu -- read-only HBM streaming kernels: the measured ceiling that
+// the weight-only GEMM's bandwidth is normalised to.
+//
+// The v100-skinny pages quote their kernels' effective bandwidth as a
+// fraction of the GPU's read-only limit (aiwitness.kr post, section
+// "내가 실제로 만든 것": 879 GB/s on V100), not of a copy.  A GEMM whose
+// weights dominate its traffic only reads, so its ceiling is a pure read
+// stream.  Two ways of reading are measured, and the faster one is the
+// ceiling:
+//   * method 0: every thread streams 16-byte loads (ld.global.nc with no L1
+//     allocation), eight in flight, over a grid-stride loop;
+//   * method 1: one CTA per SM streams contiguous 36 KB blocks into a ring
+//     of shared-memory slots with bulk copies (the TMA engine), as the GEMM
+//     does, and discards them.
+// Neither writes anything but a never-taken sink store that keeps the loads
+// alive.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/skinny.h"
+#include "ptx.cuh"
+
+namespace skinny {
+namespace {
+
+constexpr int kLdgThreads = 512;
+constexpr int kLdgBlocksPerSm = 4;
+constexpr int kLdgUnroll = 8;
+constexpr int kBulkBytes = 36864;   // one NVFP4 tile
+constexpr int kBulkStages = 4;
+constexpr uint64_t kBulkWaitNs = 1000000000ull;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__global__ void __launch_bounds__(kLdgThreads) read_ldg(const uint4* __restrict__ buf, size_t n16,
+                                                       unsigned* sink)
+{
+    uint32_t acc = 0;
+    size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (; i + (kLdgUnroll - 1) * stride < n16; i += kLdgUnroll * stride) {
+        uint4 v[kLdgUnroll];
+#pragma unroll
+        for (int u = 0; u < kLdgUnroll; ++u) v[u] = ld_stream(buf + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < kLdgUnroll; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+    }
+    for (; i < n16; i += stride) {
+        const uint4 v = ld_stream(buf + i);
+        acc ^= v.x ^ v.y ^ v.z ^ v.w;
+    }
+    if (acc == 0x9E3779B9u && sink) *sink = acc;
+}
+
+// CTA b streams blocks [b*B/P, (b+1)*B/P) of the B whole blocks.  Thread 0
+// alone works: it keeps kBulkStages copies in flight and re-issues a slot as
+// soon as its copy has landed.  Every wait is bounded; after a give-up no
+// new copy is issued but the ones in flight are still waited for.
+__global__ void __launch_bounds__(32) read_bulk(const uint8_t* buf, int blocks)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kBulkStages * kBulkBytes);
+    const int P = gridDim.x, b = blockIdx.x;
+    const int t0 = (int)((int64_t)b * blocks / P), t1 = (int)((int64_t)(b + 1) * blocks / P);
+    const int n = t1 - t0;
+    if (threadIdx.x != 0) return;
+    for (int s = 0; s < kBulkStages; ++s) ptx::mbar_init(&full[s], 1);
+    ptx::fence_mbar_init();
+    const uint64_t pol = ptx::policy_evict_first();
+    auto issue = [&](int q) {
+        const int s = q % kBulkStages;
+        ptx::mbar_arrive_expect_tx(&full[s], kBulkBytes);
+        ptx::bulk_g2s(smem + (size_t)s * kBulkBytes, buf + (size_t)(t0 + q) * kBulkBytes, kBulkBytes, &full[s], pol);
+    };
+    for (int q = 0; q < kBulkStages && q < n; ++q) issue(q);
+    bool ok = true;
+    for (int q = 0; q < n; ++q) {
+        if (!ptx::mbar_wait(&full[q % kBulkStages], (q / kBulkStages) & 1, kBulkWaitNs)) ok = false;
+        if (ok && q + kBulkStages < n) issue(q + kBulkStages);
+    }
+}
+
+}  // namespace
+}  // namespace skinny
+
+using namespace skinny;
+
+extern "C" int skinny_stream_read(const void* buf, size_t bytes, int method, unsigned* sink, void* stream)
+{
+    if (!buf || bytes < 16 || (method != 0 && method != 1)) return SKINNY_ERR_INVALID_ARG;
+    if ((uintptr_t)buf % 16 != 0) return SKINNY_ERR_ALIGNMENT;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return SKINNY_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (method == 0) {
+        read_ldg<<<sms * kLdgBlocksPerSm, kLdgThreads, 0, st>>>(static_cast<const uint4*>(buf), bytes / 16, sink);
+    } else {
+        const int smem = kBulkStages * kBulkBytes + 8 * kBulkStages;
+        if (cudaFuncSetAttribute(read_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return SKINNY_ERR_CUDA;
+        const size_t blocks = bytes / kBulkBytes;
+        if (blocks == 0 || blocks >= (size_t(1) << 31)) return SKINNY_ERR_UNSUPPORTED;
+        read_bulk<<<sms, 32, smem, st>>>(static_cast<const uint8_t*>(buf), (int)blocks);
+    }
+    return cudaGetLastError() == cudaSuccess ? SKINNY_OK : SKINNY_ERR_CUDA;
+}

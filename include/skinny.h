@@ -328,6 +328,25 @@ size_t skinny_static_workspace_capacity(void);
  * SKINNY_ERR_INVALID_ARG (null addr) or SKINNY_ERR_CUDA. */
 int skinny_debug_static_workspace_address(void** addr);
 
+/* ------------------------------------------------------------------------
+ * Measurement.
+ * ---------------------------------------------------------------------- */
+
+/* Read `bytes` of device memory once, as fast as this GPU allows, and
+ * discard them: the read-only bandwidth ceiling that the GEMMs' effective
+ * bandwidth is normalised to (the v100-skinny pages quote their kernels
+ * against the read-only limit: aiwitness.kr post, section "내가 실제로 만든
+ * 것").  method 0: 16-byte loads from every thread (ld.global.nc, no L1
+ * allocation), 8 in flight per thread; it reads bytes rounded down to a
+ * multiple of 16.  method 1: one CTA per SM, contiguous 36 KB bulk copies
+ * into a 4-slot shared-memory ring, as the GEMMs stream their weights; it
+ * reads bytes rounded down to a multiple of 36864.  Asynchronous on
+ * `stream`; time it with events.  `sink` (device, may be NULL) is written
+ * only if the loaded data XOR to a fixed constant, which keeps the loads
+ * live.  Returns SKINNY_OK, INVALID_ARG (null buf, bytes < 16, bad method),
+ * ALIGNMENT (buf not 16-byte aligned), UNSUPPORTED or CUDA. */
+int skinny_stream_read(const void* buf, size_t bytes, int method, unsigned* sink, void* stream);
+
 /* Device-side error word of the current device.  Every wait inside the
  * kernels is bounded; a wait that gives up sets a bit here instead of
  * hanging (1 = wait for a weight tile, 2 = wait for a free ring slot,
