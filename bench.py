@@ -280,7 +280,7 @@ def clone_weight(w):
     return sk.PackedFP8(w.codes.clone(), w.channel_scale, w.N, w.K)
 
 
-def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, trials: int = 10):
+def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, trials: int = 10, passes=PASSES):
     """Device time of one launch of each GEMM of the step, [pass][gemm] in us:
     the median and the best of `trials` trials.
 
@@ -293,14 +293,14 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, tri
     import torch
 
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
-    out = np.zeros((len(PASSES), len(si.MIXED_LAYER)))
+    out = np.zeros((len(passes), len(si.MIXED_LAYER)))
     best = np.zeros_like(out)
     stream = torch.cuda.Stream()
     for i, spec in enumerate(si.MIXED_LAYER):
         base = weights[0][i]
         n_copy = max(COPIES, int(np.ceil(4 * l2 / weight_bytes(spec))))
         copies = [weights[c][i] for c in range(COPIES)] + [clone_weight(base) for _ in range(n_copy - COPIES)]
-        for pi, M in enumerate(PASSES):
+        for pi, M in enumerate(passes):
             stream.wait_stream(torch.cuda.current_stream())
             with torch.cuda.stream(stream):
                 launch_one(ys[M][i], xs[M][i], copies[0], ws)
@@ -327,6 +327,27 @@ def per_launch_us(weights, xs, ys, ws, launches: int = 30, replays: int = 3, tri
         del copies
     torch.cuda.empty_cache()
     return out, best
+
+
+def m16_per_gemm(weights, ws, dur_us, peak):
+    """Each GEMM of the step at M = 16 (two MMA token blocks), timed like the
+    M = 1 and M = 8 launches, next to its M = 8 time."""
+    import torch
+
+    dev = ws.device
+    xs = {16: [torch.from_numpy(si.activations(16, s.K, seed=0, cfg_id=si.MIXED_CFG_ID, tensor_id=200 + i)).to(dev)
+               for i, s in enumerate(si.MIXED_LAYER)]}
+    ys = {16: [torch.empty((16, s.N), dtype=torch.float32 if s.out == "f32" else torch.float16, device=dev)
+               for s in si.MIXED_LAYER]}
+    med, best = per_launch_us(weights, xs, ys, ws, passes=(16,))
+    rows = []
+    for i, spec in enumerate(si.MIXED_LAYER):
+        b16, b8 = gemm_bytes(spec, 16), gemm_bytes(spec, 8)
+        g16, g8 = b16 / med[0, i] / 1e3, b8 / float(dur_us[PASSES.index(8), i]) / 1e3
+        rows.append({"gemm": spec.name, "fmt": spec.fmt, "us": round(float(med[0, i]), 3),
+                     "us_best": round(float(best[0, i]), 3), "GB/s": round(g16, 1), "frac": round(g16 / peak, 4),
+                     "GB/s_vs_M8": round(g16 / g8, 4)})
+    return rows
 
 
 def grouped_attention_us(weights, xs, ys, ws, peak, launches: int = 30, replays: int = 3, trials: int = 10):
@@ -787,6 +808,7 @@ def main(argv=None):
     dur_us, best_us = per_launch_us(weights, xs, ys, ws)
     ro_peak, ro_methods = read_only_ceiling(dev)
     grouped = grouped_attention_us(weights, xs, ys, ws, peak)
+    m16 = m16_per_gemm(weights, ws, dur_us, peak)
     fused = fused_epilogues_us(dev)
 
     for i in range(args.warmup):
@@ -803,6 +825,17 @@ def main(argv=None):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    # Ten more trials of the same K steps (not part of the value): their median
+    # and best show how steady the timed region was.
+    trial_ms = []
+    for _ in range(10):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for i in range(args.steps):
+            graphs[i % COPIES].replay()
+        t1.record()
+        torch.cuda.synchronize()
+        trial_ms.append(t0.elapsed_time(t1) / args.steps)
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert sk.device_error(clear=True) == 0, "a device-side wait gave up"
 
@@ -848,8 +881,12 @@ def main(argv=None):
                                "the timed region; achieved = algorithmic bytes / time summed over the step's NVFP4 "
                                "launches"},
         "sum_launch_us": round(float(dur_us.sum()), 2),
+        "step_trials": {"ms_per_step_median": round(float(np.median(trial_ms)), 5),
+                        "ms_per_step_best": round(float(np.min(trial_ms)), 5), "trials": len(trial_ms),
+                        "note": "10 more runs of the same K steps after the timed region (not part of value)"},
         "per_gemm": per,
         "grouped_attention": grouped,
+        "per_gemm_m16": m16,
         "fused_epilogues": dict(fused, note="next rows: the per-token argmax, the SiLU*mul activation and the "
                                             "residual add fused into the GEMM epilogue, each next to the plain "
                                             "GEMM it replaces; per-launch device time, not part of the step"),

@@ -149,6 +149,7 @@ struct Member {
     float out_scale;              // NVFP4 per-tensor scale (FP8: unused, the channel scales apply)
     int N;
     int g_begin;                  // first row tile of this GEMM in the launch's tile sequence
+    int u_begin;                  // its first tile (g_begin * C)
 };
 
 struct Params {
@@ -171,24 +172,48 @@ struct Params {
     float* out_val;               // [M]
 };
 
-// The GEMM of the launch that owns row tile g.
-__device__ __forceinline__ int member_of(const Params& p, int g)
+// The GEMM of the launch that owns row tile g (member_of_row) or tile u
+// (member_of_tile).  A launch of one GEMM (GR = false) has member 0 only,
+// resolved at compile time, so its kernels carry no lookup at all.
+template <bool GR>
+__device__ __forceinline__ int member_of_row(const Params& p, int g)
 {
-    int m = p.n_members - 1;
-    while (m > 0 && g < p.mem[m].g_begin) --m;
-    return m;
+    if constexpr (!GR) {
+        return 0;
+    } else {
+        int m = p.n_members - 1;
+        while (m > 0 && g < p.mem[m].g_begin) --m;
+        return m;
+    }
 }
 
-// CTA b of P takes quanta [b*UQ/P, (b+1)*UQ/P) of the UQ = U/Q quanta.
-__host__ __device__ __forceinline__ int range_start(int b, int P, int UQ, int Q)
+template <bool GR>
+__device__ __forceinline__ int member_of_tile(const Params& p, int u)
 {
-    return (int)(((int64_t)b * UQ) / P) * Q;
+    if constexpr (!GR) {
+        return 0;
+    } else {
+        int m = p.n_members - 1;
+        while (m > 0 && u < p.mem[m].u_begin) --m;
+        return m;
+    }
+}
+
+// CTA b of P takes quanta [range_start(b), range_start(b+1)) of the UQ = U/Q
+// quanta: with q = UQ / P and r = UQ % P, the first r CTAs take q + 1 quanta
+// and the others q.  CTAs are dispatched roughly in blockIdx order as SMs
+// free up, so the CTAs that start last get the shorter ranges.  32-bit
+// arithmetic only: b * q <= UQ < 2^31.
+__host__ __device__ __forceinline__ int range_start(int b, int q, int r, int Q)
+{
+    return (b * q + (b < r ? b : r)) * Q;
 }
 
 // The CTA whose range holds tile u (inverse of range_start).
-__host__ __device__ __forceinline__ int owner_of(int u, int P, int UQ, int Q)
+__host__ __device__ __forceinline__ int owner_of(int u, int q, int r, int Q)
 {
-    return (int)((((int64_t)(u / Q) + 1) * P - 1) / UQ);
+    const int uq = u / Q, edge = r * (q + 1);
+    return uq < edge ? uq / (q + 1) : r + (uq - edge) / q;
 }
 
 // This CTA's range and the contributors of the row tiles at its two ends
@@ -205,15 +230,16 @@ struct Sched {
 __host__ __device__ __forceinline__ Sched make_sched(const Params& p, int b, int P)
 {
     const int UQ = p.U / p.Q;
+    const int q = UQ / P, r = UQ % P;   // P <= UQ, so q >= 1
     Sched s;
     s.b = b;
-    const int u_begin = range_start(b, P, UQ, p.Q);
-    s.n_units = range_start(b + 1, P, UQ, p.Q) - u_begin;
+    const int u_begin = range_start(b, q, r, p.Q);
+    s.n_units = range_start(b + 1, q, r, p.Q) - u_begin;
     s.u_last = u_begin + s.n_units - 1;
     s.first_g = u_begin / p.C;
     s.last_g = s.u_last / p.C;
-    s.first_owner = owner_of(s.first_g * p.C, P, UQ, p.Q);
-    s.last_owner = owner_of(s.last_g * p.C + p.C - 1, P, UQ, p.Q);
+    s.first_owner = owner_of(s.first_g * p.C, q, r, p.Q);
+    s.last_owner = owner_of(s.last_g * p.C + p.C - 1, q, r, p.Q);
     return s;
 }
 
@@ -252,30 +278,24 @@ __device__ __forceinline__ int argmax_key_row(unsigned long long key) { return (
 // One warp's slice of a finished row tile: strip `strip`, rows gid + 8h,
 // tokens tok0 + 2t and tok0 + 2t + 1 of this lane (v[0], v[1]; res[0],
 // res[1] the residual of those outputs when the GEMM adds one).  Called by
-// all 32 lanes.
-template <int FMT>
+// all 32 lanes.  With the fused argmax the outputs only update this lane's
+// running best keys (best[0], best[1]); they are reduced across the CTA once,
+// at the end of the kernel.
+template <int FMT, bool GR>
 __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], const float (&res)[2], int g,
-                                         int strip, int h, int lane, int tok0)
+                                         int strip, int h, int lane, int tok0, unsigned long long (&best)[2])
 {
     const int gid = lane >> 2, t = lane & 3;
-    const Member& mb = p.mem[member_of(p, g)];
+    const Member& mb = p.mem[member_of_row<GR>(p, g)];
     const int n = (g - mb.g_begin) * kTileRows + strip * kStripRows + gid + 8 * h;
     const float sc = (FMT == SKINNY_FMT_NVFP4) ? mb.out_scale : (n < mb.N ? mb.channel_scale[n] : 0.f);
     if (p.argmax) {
-        // The warp's best (value, row) per token: lanes with the same t hold
-        // the same two tokens for eight rows; one shared-memory atomic per
-        // token per warp, one global atomic per token per CTA (at the end).
         // The value is the one the FP32-output GEMM would store.
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int m = tok0 + 2 * t + e;
-            unsigned long long key = (n < mb.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
-#pragma unroll
-            for (int d = 4; d < 32; d <<= 1) {
-                const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, d);
-                key = o > key ? o : key;
-            }
-            if (gid == 0 && key != 0ull) atomicMax(&s_argmax_best[m], key);
+            const unsigned long long key = (n < mb.N && m < p.M) ? argmax_key(v[e] * sc, n) : 0ull;
+            best[e] = key > best[e] ? key : best[e];
         }
         return;
     }
@@ -340,12 +360,12 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[NB][2], int 
 // gid + 8h, tokens 8nb + 2t + e), loaded as soon as the CTA knows that it
 // finishes the row tile, so that the loads overlap the exchange and the
 // split-K wait instead of stalling the epilogue.  Zero where there is none.
-template <int NB>
+template <int NB, bool GR>
 __device__ __forceinline__ void load_residual(const Params& p, int g, int strip, int h, int lane,
                                               float (&res)[NB][2])
 {
     const int gid = lane >> 2, t = lane & 3;
-    const Member& mb = p.mem[member_of(p, g)];
+    const Member& mb = p.mem[member_of_row<GR>(p, g)];
     const int n = (g - mb.g_begin) * kTileRows + strip * kStripRows + gid + 8 * h;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -364,15 +384,17 @@ __device__ __forceinline__ void load_residual(const Params& p, int g, int strip,
 // The finished outputs of row tile g (this warp's slice) go to y, to the
 // fused argmax, or through the fused SiLU*mul.  Called by every warp of the
 // CTA together.
-template <int FMT, int NB>
+template <int FMT, int NB, bool GR>
 __device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2], const float (&res)[NB][2], int g,
-                                       int strip, int h, int lane, uint8_t* smem)
+                                       int strip, int h, int lane, uint8_t* smem,
+                                       unsigned long long (&best)[NB][2])
 {
-    if (FMT == SKINNY_FMT_NVFP4 && p.silu_mul) {
+    if (FMT == SKINNY_FMT_NVFP4 && !GR && p.silu_mul) {
         silu_mul_epilogue<FMT, NB>(p, v, g, strip, h, lane, smem);
     } else {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) epilogue<FMT>(p, v[nb], res[nb], g, strip, h, lane, kBlockTokens * nb);
+        for (int nb = 0; nb < NB; ++nb)
+            epilogue<FMT, GR>(p, v[nb], res[nb], g, strip, h, lane, kBlockTokens * nb, best[nb]);
     }
 }
 
@@ -390,9 +412,9 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2],
 // Which case applies is the same for every warp of the CTA, so the barriers
 // of the exchange and of the fused epilogues are reached by all of them.
 // With two token blocks every lane carries both blocks' sums (NB pairs).
-template <int FMT, int NB>
+template <int FMT, int NB, bool GR>
 __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int c_first, int c_last, int parity,
-                      uint8_t* smem, int b, int warp, int lane)
+                      uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2])
 {
     using S = Smem<FMT, NB>;
     float4* xchg = reinterpret_cast<float4*>(smem + S::kXchgOff) + parity * S::kXchgFloat4;
@@ -400,7 +422,7 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
     const int sq = kq >> 1, h = kq & 1;          // this warp finishes strip 2sp+sq, rows gid+8h
     const int strip = 2 * sp + sq;
     float res[NB][2];
-    if (c_first == c_last || b == c_last) load_residual<NB>(p, g, strip, h, lane, res);
+    if (c_first == c_last || b == c_last) load_residual<NB, GR>(p, g, strip, h, lane, res);
 #pragma unroll
     for (int q = 0; q < 2; ++q)
 #pragma unroll
@@ -420,7 +442,7 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
             tot[nb][1] += h ? v.w : v.y;
         }
     if (c_first == c_last) {
-        finish<FMT, NB>(p, tot, res, g, strip, h, lane, smem);
+        finish<FMT, NB, GR>(p, tot, res, g, strip, h, lane, smem, best);
         return;
     }
     uint2* const mine = p.partials + ((b * kConsumerWarps + warp) * 32 + lane) * NB;
@@ -481,15 +503,15 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
         sum[nb][0] += tot[nb][0];
         sum[nb][1] += tot[nb][1];
     }
-    finish<FMT, NB>(p, sum, res, g, strip, h, lane, smem);
+    finish<FMT, NB, GR>(p, sum, res, g, strip, h, lane, smem, best);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.
-template <int FMT, int NB>
+template <int FMT, int NB, bool GR>
 __device__ __forceinline__ void issue_stage(const Params& p, uint8_t* smem, uint64_t* full, int s, int u)
 {
-    const Member& mb = p.mem[member_of(p, u / p.C)];
-    const uint8_t* src = mb.codes + (size_t)(u - mb.g_begin * p.C) * Tile<FMT>::kBytes;
+    const Member& mb = p.mem[member_of_tile<GR>(p, u)];
+    const uint8_t* src = mb.codes + (size_t)(GR ? u - mb.u_begin : u) * Tile<FMT>::kBytes;
     ptx::mbar_arrive_expect_tx(&full[s], Tile<FMT>::kBytes);
     ptx::bulk_g2s(smem + s * Smem<FMT, NB>::kStageBytes, src, Tile<FMT>::kBytes, &full[s],
                   ptx::policy_evict_first());
@@ -616,7 +638,7 @@ struct Consumer {
 // token block the activations of the next tile are fetched one tile ahead
 // into ping-pong registers; with two there is no room for a second set, and
 // each tile's activations are fetched as the tile begins (before its wait).
-template <int FMT, int NB>
+template <int FMT, int NB, bool GR>
 __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, const Sched& sc, int warp,
                         int lane)
 {
@@ -652,17 +674,21 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     int g = sc.last_g, c = sc.u_last - sc.last_g * p.C;   // tile being processed
     int nc = c;                                            // K tile whose activations are fetched next
     int ng = g;                                            // ... and its row tile
-    int nm = member_of(p, ng);                             // ... and its GEMM
+    int nm = member_of_row<GR>(p, ng);                     // ... and its GEMM
     const uint16_t* xbase = p.mem[nm].x;
     const uint32_t smem32 = ptx::smem_addr(smem);
     int* released = reinterpret_cast<int*>(smem + S::kCountOff);
+    // Fused argmax: this lane's best key per token it holds (tokens 8nb + 2t + e).
+    unsigned long long best[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) best[nb][0] = best[nb][1] = 0ull;
     // Contributors of a row tile: only the two at the ends of the range are shared.
     auto flush_g = [&](int fg) {
         float tot[2][NB][4];
         w.total(tot);
         const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
         const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
-        flush<FMT, NB>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane);
+        flush<FMT, NB, GR>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane, best);
         parity ^= 1;
     };
     auto fetch = [&](uint32_t (&dst)[2][NB][8]) {
@@ -675,7 +701,9 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     auto advance = [&]() {   // the fetch cursor moves one tile down the range
         if (nc == 0) {
             nc = p.C;
-            if (--ng < p.mem[nm].g_begin && nm > 0) xbase = p.mem[--nm].x;
+            if constexpr (GR) {
+                if (--ng < p.mem[nm].g_begin && nm > 0) xbase = p.mem[--nm].x;
+            }
         }
         --nc;
     };
@@ -706,7 +734,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
                     released[s] = 0;
                     if (i + kStages < n_units) {
                         if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
-                            issue_stage<FMT, NB>(p, smem, full, s, sc.u_last - (i + kStages));
+                            issue_stage<FMT, NB, GR>(p, smem, full, s, sc.u_last - (i + kStages));
                         else
                             atomicOr(&g_device_error, kErrEmptyWait);
                     }
@@ -749,6 +777,22 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
 
     if (n_units > 0) flush_g(cur_g);
+    if (p.argmax) {
+        // The lanes with the same t hold the same tokens for different rows:
+        // reduce over them, then one shared-memory atomic per token per warp.
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                unsigned long long key = best[nb][e];
+#pragma unroll
+                for (int d = 4; d < 32; d <<= 1) {
+                    const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, d);
+                    key = o > key ? o : key;
+                }
+                if (gid == 0 && key != 0ull) atomicMax(&s_argmax_best[kBlockTokens * nb + 2 * t + e], key);
+            }
+    }
     if (!ok && threadIdx.x == 0) {
         // After a wait gave up, tiles may still be landing in shared memory:
         // wait (bounded) for the last ring's worth before the CTA exits.
@@ -758,7 +802,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
 }
 
-template <int FMT, int NB>
+template <int FMT, int NB, bool GR>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p)
 {
     using S = Smem<FMT, NB>;
@@ -781,14 +825,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // The packed weights are read-only parameters: start streaming them
         // before the previous kernel in the stream has finished.
         for (int q = 0; q < S::kStages && q < sc.n_units; ++q)
-            issue_stage<FMT, NB>(p, smem, full, q, sc.u_last - q);
+            issue_stage<FMT, NB, GR>(p, smem, full, q, sc.u_last - q);
     }
     __syncthreads();
     // x, y, the channel scales and the workspace may belong to the previous
     // kernel: touch them only once it has completed.
     ptx::pdl_wait_prior_grid();
 
-    consume<FMT, NB>(p, smem, full, empty, sc, warp, lane);
+    consume<FMT, NB, GR>(p, smem, full, empty, sc, warp, lane);
 
     if (p.argmax) {
         // The CTA that finishes last turns the maxima into (row, value) per
@@ -823,6 +867,14 @@ struct DeviceState {
 static std::mutex g_mu;
 static DeviceState g_dev[kMaxDevices];
 
+// Raise one kernel's dynamic shared-memory limit to what it uses; true on failure.
+template <int FMT, int NB, bool GR>
+static bool set_smem()
+{
+    return cudaFuncSetAttribute(gemm_kernel<FMT, NB, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Smem<FMT, NB>::kBytes) != cudaSuccess;
+}
+
 // SM count of the current device; sets the kernels' shared-memory limit once.
 static int current_device(int* sms)
 {
@@ -834,14 +886,9 @@ static int current_device(int* sms)
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             return SKINNY_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_NVFP4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_NVFP4, 1>::kBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_NVFP4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_NVFP4, 2>::kBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_FP8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_FP8, 1>::kBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_kernel<SKINNY_FMT_FP8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Smem<SKINNY_FMT_FP8, 2>::kBytes) != cudaSuccess)
+        if (set_smem<SKINNY_FMT_NVFP4, 1, false>() || set_smem<SKINNY_FMT_NVFP4, 2, false>() ||
+            set_smem<SKINNY_FMT_NVFP4, 1, true>() || set_smem<SKINNY_FMT_NVFP4, 2, true>() ||
+            set_smem<SKINNY_FMT_FP8, 1, false>() || set_smem<SKINNY_FMT_FP8, 2, false>())
             return SKINNY_ERR_CUDA;
         d.sms = n;
         d.ready = true;
@@ -948,8 +995,17 @@ static int launch(Params p, int64_t G, int64_t K, void* workspace, size_t worksp
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2> : gemm_kernel<FMT, 1>, p) != cudaSuccess)
-        return SKINNY_ERR_CUDA;
+    cudaError_t e;
+    if constexpr (FMT == SKINNY_FMT_NVFP4) {
+        if (p.n_members > 1)
+            e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, true> : gemm_kernel<FMT, 1, true>, p);
+        else
+            e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, false> : gemm_kernel<FMT, 1, false>, p);
+    } else {
+        if (p.n_members != 1) return SKINNY_ERR_UNSUPPORTED;
+        e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, false> : gemm_kernel<FMT, 1, false>, p);
+    }
+    if (e != cudaSuccess) return SKINNY_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SKINNY_OK : SKINNY_ERR_CUDA;
 }
 
@@ -1125,6 +1181,8 @@ extern "C" int skinny_nvfp4_gemm_grouped(const skinny_nvfp4_group_member* member
     p.M = M;
     p.K = (int)K;
     p.out_f32 = out_dtype == SKINNY_OUT_F32;
+    const int C = (int)((K + kTileK - 1) / kTileK);
+    for (int m = 0; m < count; ++m) p.mem[m].u_begin = p.mem[m].g_begin * C;   // < 2^31: checked by make_plan
     return launch<SKINNY_FMT_NVFP4>(p, G, K, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 

@@ -10,6 +10,8 @@ kernel's split-K fixup relies on:
     reaches that row tile LAST in its backwards walk (its first row tile),
     while every other contributor reaches it first or holds nothing else;
   * so a finisher only ever waits for lower-numbered CTAs;
+  * the ranges differ by at most one quantum, longest first (the CTAs that
+    are dispatched first take the longer ranges);
   * without split-K every row tile has exactly one contributor.
 """
 import ctypes
@@ -69,6 +71,11 @@ def test_schedule_properties(N, K, sms, split):
             assert last_g[c] == g
         assert np.all(cs[:-1] < c_last)                     # waits only on lower CTAs
     assert np.all(publishes <= 1)
+    # CTAs dispatched first (lower numbers) take the longer ranges: lengths
+    # differ by at most one quantum and never increase with the CTA number
+    quantum = 1 if split else C
+    assert n_units.max() - n_units.min() <= quantum
+    assert np.all(np.diff(n_units) <= 0)
 
 
 def test_schedule_rejects_bad_arguments():
