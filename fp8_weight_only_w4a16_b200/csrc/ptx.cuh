@@ -148,6 +148,9 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Hint: bring the cache line holding p into L1 (no register written).
+__device__ __forceinline__ void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
 // Shared-memory loads by 32-bit shared-window address (no generic-address
 // arithmetic).  The "memory" clobber keeps them after the mbarrier wait that
 // made the data visible.

@@ -698,6 +698,15 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
             for (int nb = 0; nb < NB; ++nb)
                 load_b(xbase + xoff[nb], xvalid[nb], nc * kTileK + kb_lane + u * kChunkK, p.K, dst[u][nb]);
     };
+    auto prefetch_l1 = [&]() {   // the lines `fetch` will read at the cursor
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int kb = nc * kTileK + kb_lane + u * kChunkK;
+                if (xvalid[nb] && kb < p.K) ptx::prefetch_l1(xbase + xoff[nb] + kb);
+            }
+    };
     auto advance = [&]() {   // the fetch cursor moves one tile down the range
         if (nc == 0) {
             nc = p.C;
@@ -768,10 +777,14 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         }
         if (i < n_units) step(i, bx[0], bx[1]);
     } else {
+        // No room for a second set of activation registers: fetch each tile's
+        // activations as the tile begins, and pull the next tile's lines into
+        // L1 meanwhile so that fetch hits L1.
         uint32_t bx[2][NB][8];
         for (int i = 0; i < n_units; ++i) {
             fetch(bx);
             advance();
+            if (i + 1 < n_units) prefetch_l1();
             body(i, bx);
         }
     }
