@@ -54,21 +54,36 @@
 
 namespace skinny {
 
-// 16 warps, all consumers.  Warp w handles strip pair sp = w % 4 (strips
-// 2sp, 2sp+1) and chunk pair kq = w / 4 (chunks 2kq, 2kq+1) of every tile, so
-// warps sp, sp+4, sp+8, sp+12 hold the four K quarters of the same 32 rows
-// and add them at flush time.  There is no producer warp: thread 0 issues
-// the first stages, and each later stage is issued by the warp that is last
-// to release the ring slot it refills (so 16 warps keep 4 warps per SM
-// sub-partition and up to 128 registers each).
-constexpr int kConsumerWarps = 16;
-constexpr int kStripPairs = kStrips / 2;                       // 4
-constexpr int kChunkPairs = kConsumerWarps / kStripPairs;      // 4
+// All warps are consumers.  A warp handles kStripsPerWarp consecutive strips
+// (strip group sg = w % kStripGroups) and the chunk pair kq = w / kStripGroups
+// (chunks 2kq, 2kq+1) of every tile, so the kChunkPairs warps of a strip
+// group hold the four K quarters of the same rows and add them at flush
+// time.  There is no producer warp: thread 0 issues the first stages, and
+// each later stage is issued by the warp that is last to release the ring
+// slot it refills.
+#ifndef SKINNY_STRIPS_PER_WARP
+#define SKINNY_STRIPS_PER_WARP 2
+#endif
+constexpr int kStripsPerWarp = SKINNY_STRIPS_PER_WARP;          // 2: 16 warps, 4: 8 warps
+constexpr int kStripGroups = kStrips / kStripsPerWarp;
+constexpr int kChunkPairs = kChunks / 2;                        // 4
+constexpr int kConsumerWarps = kStripGroups * kChunkPairs;
 constexpr int kThreads = kConsumerWarps * 32;
+// (strip, row half) pairs of a strip group finished by each of its warps.
+constexpr int kFinishPerWarp = kStripsPerWarp / 2;
+static_assert(kStripsPerWarp == 2 || kStripsPerWarp == 4, "2 or 4 strips per warp");
+
+// The f-th (strip, row half) pair that warp (sg, kq) finishes: strip
+// kStripsPerWarp * sg + pi / 2, rows gid + 8 * (pi % 2), pi = kq * kFinishPerWarp + f.
+__host__ __device__ __forceinline__ int finish_strip(int sg, int kq, int f)
+{
+    return kStripsPerWarp * sg + (kq * kFinishPerWarp + f) / 2;
+}
+__host__ __device__ __forceinline__ int finish_half(int kq, int f) { return (kq * kFinishPerWarp + f) % 2; }
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 constexpr int kMaxDevices = 64;
 
-static_assert(kChunkPairs * 2 == kChunks, "two chunks per consumer warp");
+
 
 // Named barrier id of the 16 consumer warps (0 is __syncthreads).
 constexpr uint32_t kBarConsumers = 1;
@@ -123,7 +138,7 @@ struct Smem {
     static constexpr int kStages = (FMT == SKINNY_FMT_FP8 && NB == 2) ? 2 : Tile<FMT>::kStages;
     static constexpr int kStageBytes = Tile<FMT>::kBytes;
     static constexpr int kXchgOff = kStages * kStageBytes;
-    static constexpr int kXchgFloat4 = kConsumerWarps * 2 * NB * 32;   // one parity
+    static constexpr int kXchgFloat4 = kConsumerWarps * kStripsPerWarp * NB * 32;   // one parity
     static constexpr int kXchgBytes = 2 * kXchgFloat4 * 16;
     static constexpr int kBarOff = kXchgOff + kXchgBytes;
     static constexpr int kCountOff = kBarOff + 2 * kStages * 8;   // int released[kStages]
@@ -324,26 +339,29 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], c
 // so the tile yields outputs j = 64g + 0..63 of every token:
 // y[m][j] = silu(gate) * up, silu(z) = z / (1 + e^-z), in FP32.
 template <int FMT, int NB>
-__device__ void silu_mul_epilogue(const Params& p, const float (&v)[NB][2], int g, int strip, int h, int lane,
-                                  uint8_t* smem)
+__device__ void silu_mul_epilogue(const Params& p, const float (&v)[kFinishPerWarp][NB][2], int g, int sg, int kq,
+                                  int lane, uint8_t* smem)
 {
     constexpr int kTok = kBlockTokens * NB;
     float* act = reinterpret_cast<float*>(smem + Smem<FMT, NB>::kActOff);   // [128 rows][kTok tokens]
     const int gid = lane >> 2, t = lane & 3;
-    const int r = strip * kStripRows + gid + 8 * h;
     const Member& mb = p.mem[0];   // the fused SiLU*mul runs one GEMM per launch
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        act[r * kTok + kBlockTokens * nb + 2 * t] = v[nb][0] * mb.out_scale;
-        act[r * kTok + kBlockTokens * nb + 2 * t + 1] = v[nb][1] * mb.out_scale;
+    for (int f = 0; f < kFinishPerWarp; ++f) {
+        const int r = finish_strip(sg, kq, f) * kStripRows + gid + 8 * finish_half(kq, f);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            act[r * kTok + kBlockTokens * nb + 2 * t] = v[f][nb][0] * mb.out_scale;
+            act[r * kTok + kBlockTokens * nb + 2 * t + 1] = v[f][nb][1] * mb.out_scale;
+        }
     }
     ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    const int jl = threadIdx.x % 64;                                  // 64 outputs x 8 tokens per pass
+    const int jl = threadIdx.x % 64;                     // 64 outputs x kThreads/64 tokens per pass
     const int F = mb.N / 2, j = g * 64 + jl;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        const int m = threadIdx.x / 64 + kBlockTokens * nb;
+    for (int pass = 0; pass < kTok / (kThreads / 64); ++pass) {
+        const int m = threadIdx.x / 64 + (kThreads / 64) * pass;
         if (m < p.M && j < F) {
             const float gate = act[jl * kTok + m], up = act[(64 + jl) * kTok + m];
             const float val = gate / (1.f + expf(-gate)) * up;
@@ -385,24 +403,27 @@ __device__ __forceinline__ void load_residual(const Params& p, int g, int strip,
 // fused argmax, or through the fused SiLU*mul.  Called by every warp of the
 // CTA together.
 template <int FMT, int NB, bool GR>
-__device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2], const float (&res)[NB][2], int g,
-                                       int strip, int h, int lane, uint8_t* smem,
-                                       unsigned long long (&best)[NB][2])
+__device__ __forceinline__ void finish(const Params& p, const float (&v)[kFinishPerWarp][NB][2],
+                                       const float (&res)[kFinishPerWarp][NB][2], int g, int sg, int kq, int lane,
+                                       uint8_t* smem, unsigned long long (&best)[NB][2])
 {
     if (FMT == SKINNY_FMT_NVFP4 && !GR && p.silu_mul) {
-        silu_mul_epilogue<FMT, NB>(p, v, g, strip, h, lane, smem);
+        silu_mul_epilogue<FMT, NB>(p, v, g, sg, kq, lane, smem);
     } else {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-            epilogue<FMT, GR>(p, v[nb], res[nb], g, strip, h, lane, kBlockTokens * nb, best[nb]);
+        for (int f = 0; f < kFinishPerWarp; ++f)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                epilogue<FMT, GR>(p, v[f][nb], res[f][nb], g, finish_strip(sg, kq, f), finish_half(kq, f), lane,
+                                  kBlockTokens * nb, best[nb]);
     }
 }
 
 // Finish (or contribute to) row tile g, whose K range CTAs c_first..c_last
-// share.  The four warps of a strip pair (sp, sp+4, sp+8, sp+12) hold the
-// four K quarters of strips 2sp and 2sp+1; through shared memory each of them
-// takes one quarter of the strip pair's outputs (strip 2sp + kq/2, rows
-// gid + 8*(kq%2)) and adds the four K quarters in order (a fixed order).
+// share.  The kChunkPairs warps of a strip group (sg, kq = 0..3) hold the four
+// K quarters of its strips; through shared memory each of them takes
+// kFinishPerWarp (strip, row half) pairs of the group's outputs and adds the
+// four K quarters in order (a fixed order).
 //  * c_first == c_last: this CTA covered all of K; finish the outputs
 //    (store y, or the fused argmax / SiLU*mul).
 //  * this CTA is not c_last: publish the partial sums in this CTA's slot.
@@ -413,70 +434,85 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[NB][2],
 // of the exchange and of the fused epilogues are reached by all of them.
 // With two token blocks every lane carries both blocks' sums (NB pairs).
 template <int FMT, int NB, bool GR>
-__device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int c_first, int c_last, int parity,
-                      uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2])
+__device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4], int g, int c_first, int c_last,
+                      int parity, uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2])
 {
     using S = Smem<FMT, NB>;
+    constexpr int F = kFinishPerWarp;
     float4* xchg = reinterpret_cast<float4*>(smem + S::kXchgOff) + parity * S::kXchgFloat4;
-    const int sp = warp % kStripPairs, kq = warp / kStripPairs;
-    const int sq = kq >> 1, h = kq & 1;          // this warp finishes strip 2sp+sq, rows gid+8h
-    const int strip = 2 * sp + sq;
-    float res[NB][2];
-    if (c_first == c_last || b == c_last) load_residual<NB, GR>(p, g, strip, h, lane, res);
+    const int sg = warp % kStripGroups, kq = warp / kStripGroups;
 #pragma unroll
-    for (int q = 0; q < 2; ++q)
+    for (int q = 0; q < kStripsPerWarp; ++q)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
-            xchg[((warp * 2 + q) * NB + nb) * 32 + lane] =
+            xchg[((warp * kStripsPerWarp + q) * NB + nb) * 32 + lane] =
                 make_float4(acc[q][nb][0], acc[q][nb][1], acc[q][nb][2], acc[q][nb][3]);
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    float tot[NB][2];
+    float res[F][NB][2];
+    if (c_first == c_last || b == c_last) {
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) tot[nb][0] = tot[nb][1] = 0.f;
+        for (int f = 0; f < F; ++f)
+            load_residual<NB, GR>(p, g, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
+    }
+    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
+    float tot[F][NB][2];
+#pragma unroll
+    for (int f = 0; f < F; ++f)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) tot[f][nb][0] = tot[f][nb][1] = 0.f;
 #pragma unroll
     for (int k = 0; k < kChunkPairs; ++k)
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-            const float4 v = xchg[(((k * kStripPairs + sp) * 2 + sq) * NB + nb) * 32 + lane];
-            tot[nb][0] += h ? v.z : v.x;
-            tot[nb][1] += h ? v.w : v.y;
-        }
+        for (int f = 0; f < F; ++f)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                const int q = finish_strip(sg, kq, f) - kStripsPerWarp * sg;
+                const float4 v = xchg[(((k * kStripGroups + sg) * kStripsPerWarp + q) * NB + nb) * 32 + lane];
+                const bool hi = finish_half(kq, f) != 0;
+                tot[f][nb][0] += hi ? v.z : v.x;
+                tot[f][nb][1] += hi ? v.w : v.y;
+            }
     if (c_first == c_last) {
-        finish<FMT, NB, GR>(p, tot, res, g, strip, h, lane, smem, best);
+        finish<FMT, NB, GR>(p, tot, res, g, sg, kq, lane, smem, best);
         return;
     }
-    uint2* const mine = p.partials + ((b * kConsumerWarps + warp) * 32 + lane) * NB;
+    constexpr int kSlot = F * NB;   // uint2 per lane
+    uint2* const mine = p.partials + ((b * kConsumerWarps + warp) * 32 + lane) * kSlot;
     if (b != c_last) {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-            ptx::st_volatile_v2(mine + nb, make_uint2(encode_partial(tot[nb][0]), encode_partial(tot[nb][1])));
+        for (int f = 0; f < F; ++f)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                ptx::st_volatile_v2(mine + f * NB + nb,
+                                    make_uint2(encode_partial(tot[f][nb][0]), encode_partial(tot[f][nb][1])));
         return;
     }
     // Finisher.  The other contributors are lower-numbered CTAs; all but the
     // middle ones (whose whole range lies in g) published long ago.
-    constexpr int kBatch = 8 / NB;
-    float sum[NB][2];
+    constexpr int kBatch = 8 / kSlot;
+    float sum[F][NB][2];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = 0.f;
+    for (int f = 0; f < F; ++f)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) sum[f][nb][0] = sum[f][nb][1] = 0.f;
     bool timed_out = false;
     uint64_t t0 = 0;
     for (int c0 = c_first; c0 < c_last; c0 += kBatch) {
-        uint2 v[kBatch][NB];
-        auto slot = [&](int k) { return p.partials + (((c0 + k) * kConsumerWarps + warp) * 32 + lane) * NB; };
+        uint2 v[kBatch][kSlot];
+        auto slot = [&](int k) { return p.partials + (((c0 + k) * kConsumerWarps + warp) * 32 + lane) * kSlot; };
 #pragma unroll
         for (int k = 0; k < kBatch; ++k)
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-                v[k][nb] = (c0 + k < c_last) ? ptx::ld_volatile_v2(slot(k) + nb) : make_uint2(1u, 1u);
+            for (int e = 0; e < kSlot; ++e)
+                v[k][e] = (c0 + k < c_last) ? ptx::ld_volatile_v2(slot(k) + e) : make_uint2(1u, 1u);
         for (uint32_t it = 0;; ++it) {
             bool missing = false;
 #pragma unroll
             for (int k = 0; k < kBatch; ++k)
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    if (v[k][nb].x == 0u || v[k][nb].y == 0u) {
+                for (int e = 0; e < kSlot; ++e) {
+                    if (v[k][e].x == 0u || v[k][e].y == 0u) {
                         missing = true;
-                        v[k][nb] = ptx::ld_volatile_v2(slot(k) + nb);
+                        v[k][e] = ptx::ld_volatile_v2(slot(k) + e);
                     }
                 }
             if (!missing || timed_out) break;
@@ -490,20 +526,25 @@ __device__ void flush(const Params& p, const float (&acc)[2][NB][4], int g, int 
         for (int k = 0; k < kBatch; ++k) {
             if (c0 + k < c_last) {
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    sum[nb][0] += decode_partial(v[k][nb].x);
-                    sum[nb][1] += decode_partial(v[k][nb].y);
-                    ptx::st_volatile_v2(slot(k) + nb, make_uint2(0u, 0u));
-                }
+                for (int f = 0; f < F; ++f)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        sum[f][nb][0] += decode_partial(v[k][f * NB + nb].x);
+                        sum[f][nb][1] += decode_partial(v[k][f * NB + nb].y);
+                    }
+#pragma unroll
+                for (int e = 0; e < kSlot; ++e) ptx::st_volatile_v2(slot(k) + e, make_uint2(0u, 0u));
             }
         }
     }
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        sum[nb][0] += tot[nb][0];
-        sum[nb][1] += tot[nb][1];
-    }
-    finish<FMT, NB, GR>(p, sum, res, g, strip, h, lane, smem, best);
+    for (int f = 0; f < F; ++f)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            sum[f][nb][0] += tot[f][nb][0];
+            sum[f][nb][1] += tot[f][nb][1];
+        }
+    finish<FMT, NB, GR>(p, sum, res, g, sg, kq, lane, smem, best);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.
@@ -533,23 +574,25 @@ __device__ __forceinline__ void load_b(const uint16_t* xrow, bool valid, int kb,
     bx[4] = x1.x; bx[5] = x1.y; bx[6] = x1.z; bx[7] = x1.w;
 }
 
-// Per-warp state of the consumer loop.  A warp owns strips 2sp, 2sp+1 and K
-// chunks 2kq, 2kq+1 of every tile: four strip chunks, each with its own
-// accumulator chain per token block (hiding the tensor-core latency); the two
-// chunk accumulators of a strip are added in a fixed order when a row tile is
+// Per-warp state of the consumer loop.  A warp owns strips
+// kStripsPerWarp * sg .. + kStripsPerWarp - 1 and K chunks 2kq, 2kq+1 of every
+// tile: 2 * kStripsPerWarp strip chunks, each with its own accumulator chain
+// per token block (hiding the tensor-core latency); the two chunk
+// accumulators of a strip are added in a fixed order when a row tile is
 // flushed.
 template <int FMT, int NB>
 struct Consumer {
-    float acc[2][2][NB][4];   // [chunk parity][strip][token block][fragment]
-    uint32_t lane_codes;      // this lane's code bytes of strip 2sp, chunk 2kq, inside a tile
-    uint32_t lane_scale;      // this lane's scale word of strip 2sp, chunk 2kq (NVFP4)
+    static constexpr int Q = kStripsPerWarp;
+    float acc[2][Q][NB][4];   // [chunk parity][strip][token block][fragment]
+    uint32_t lane_codes;      // this lane's code bytes of its first strip, chunk 2kq, inside a tile
+    uint32_t lane_scale;      // this lane's scale word of its first strip, chunk 2kq (NVFP4)
 
     __device__ __forceinline__ void zero()
     {
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < Q; ++q)
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -557,10 +600,10 @@ struct Consumer {
     }
 
     // The per-strip sums of both chunks (fixed order).
-    __device__ __forceinline__ void total(float (&tot)[2][NB][4]) const
+    __device__ __forceinline__ void total(float (&tot)[Q][NB][4]) const
     {
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+        for (int q = 0; q < Q; ++q)
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -574,17 +617,17 @@ struct Consumer {
     __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][NB][8])
     {
         if constexpr (FMT == SKINNY_FMT_NVFP4) {
-            uint4 cw[2][2];
-            uint32_t s0[2][2], s8[2][2];
+            uint4 cw[2][Q];
+            uint32_t s0[2][Q], s8[2][Q];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int q = 0; q < 2; ++q)
+                for (int q = 0; q < Q; ++q)
                     cw[u][q] = ptx::lds128(tile + lane_codes + q * kNvfp4StripCodeBytes + u * 512);
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < Q; ++q) {
                     const uint32_t sc =
                         ptx::e4m3x2_to_f16x2(ptx::lds16(tile + lane_scale + q * kNvfp4StripScaleBytes + u * 64));
                     s0[u][q] = ptx::dup_lo(sc);   // scale of row gid
@@ -595,7 +638,7 @@ struct Consumer {
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
+                    for (int q = 0; q < Q; ++q) {
                         const uint32_t w = j == 0 ? cw[u][q].x : j == 1 ? cw[u][q].y : j == 2 ? cw[u][q].z : cw[u][q].w;
                         uint32_t h[4];
                         ptx::e2m1x8_to_f16x8(w, h);
@@ -606,11 +649,11 @@ struct Consumer {
                             ptx::mma_f16_16816(acc[u][q][nb], a, bx[u][nb][2 * j], bx[u][nb][2 * j + 1]);
                     }
         } else {
-            uint4 cw[2][2][2];
+            uint4 cw[2][Q][2];
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < Q; ++q) {
                     const uint32_t base = tile + lane_codes + q * kFp8StripBytes + u * 1024;
                     cw[u][q][0] = ptx::lds128(base);
                     cw[u][q][1] = ptx::lds128(base + 512);
@@ -620,7 +663,7 @@ struct Consumer {
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
+                    for (int q = 0; q < Q; ++q) {
                         const uint4& v = cw[u][q][j >> 1];
                         const uint32_t w0 = (j & 1) ? v.z : v.x, w1 = (j & 1) ? v.w : v.y;
                         uint32_t a[4];
@@ -646,16 +689,17 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     constexpr int kStages = S::kStages;
     constexpr bool kAhead = NB == 1;
     const int gid = lane >> 2, t = lane & 3;
-    const int sp = warp % kStripPairs, kq = warp / kStripPairs;
+    const int sg = warp % kStripGroups, kq = warp / kStripGroups;
     const int n_units = sc.n_units;
 
     Consumer<FMT, NB> w;
     w.zero();
+    const int strip0 = kStripsPerWarp * sg;
     if constexpr (FMT == SKINNY_FMT_NVFP4) {
-        w.lane_codes = (2 * sp) * kNvfp4StripCodeBytes + (2 * kq) * 512 + lane * 16;
-        w.lane_scale = Tile<FMT>::kScalesOff + (2 * sp) * kNvfp4StripScaleBytes + (2 * kq) * 64 + t * 16 + gid * 2;
+        w.lane_codes = strip0 * kNvfp4StripCodeBytes + (2 * kq) * 512 + lane * 16;
+        w.lane_scale = Tile<FMT>::kScalesOff + strip0 * kNvfp4StripScaleBytes + (2 * kq) * 64 + t * 16 + gid * 2;
     } else {
-        w.lane_codes = (2 * sp) * kFp8StripBytes + (2 * kq) * 1024 + lane * 16;
+        w.lane_codes = strip0 * kFp8StripBytes + (2 * kq) * 1024 + lane * 16;
         w.lane_scale = 0;
     }
     // Activations: tokens gid + 8nb, columns c*512 + (2kq + u)*64 + [16t, 16t+16),
@@ -684,7 +728,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     for (int nb = 0; nb < NB; ++nb) best[nb][0] = best[nb][1] = 0ull;
     // Contributors of a row tile: only the two at the ends of the range are shared.
     auto flush_g = [&](int fg) {
-        float tot[2][NB][4];
+        float tot[kStripsPerWarp][NB][4];
         w.total(tot);
         const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
         const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
@@ -933,7 +977,7 @@ static int make_plan(int64_t G, int64_t K, int sms, bool split, Plan* pl)
     pl->U = (int)(G * C);
     const int UQ = split ? pl->U : pl->G;
     pl->P = UQ < sms ? UQ : sms;
-    pl->partial_bytes = (size_t)sms * kConsumerWarps * 32 * 2 * sizeof(uint2);
+    pl->partial_bytes = (size_t)sms * kConsumerWarps * 32 * kFinishPerWarp * 2 * sizeof(uint2);
     pl->workspace_bytes = pl->partial_bytes + kArgmaxTailBytes;
     return SKINNY_OK;
 }
