@@ -7,17 +7,19 @@
 // their way out of HBM and become FP16 in registers for the tensor cores;
 // M=8 is the k=7 speculative-verify round).  The design here is B200-first:
 //
-//  * One persistent CTA per SM with 16 warps.  Weights stream in 128-row x
-//    512-column tiles (32 KB NVFP4 codes + 4 KB block scales, or 64 KB FP8),
-//    one tile per ring stage, each stage ONE bulk copy (the TMA engine,
-//    cp.async.bulk): a bulk copy costs its issuing thread ~150 ns, so copies
-//    must be large.  Stages are guarded by mbarriers; the warp that is last
-//    to release a slot issues its refill (no producer warp).
+//  * One persistent CTA per SM: 8 consumer warps and a producer warpgroup.
+//    Weights stream in 128-row x 512-column tiles (32 KB NVFP4 codes + 4 KB
+//    block scales, or 64 KB FP8), one tile per ring stage, each stage ONE
+//    bulk copy (the TMA engine, cp.async.bulk): a bulk copy costs its issuing
+//    thread ~150 ns, so copies must be large.  Stages are guarded by
+//    mbarriers.  One thread of the producer warpgroup refills a slot as soon
+//    as every consumer warp has released it, off the consumers' critical
+//    path; the warpgroup gives its registers to the consumers (setmaxnreg).
 //  * Programmatic dependent launch: a CTA starts streaming its first tiles
 //    while the previous kernel in the stream is still finishing, and touches
 //    x, y and the workspace only after that kernel has completed.
 //  * Activations are read by each lane straight from x (L1-cached), one tile
-//    ahead of use; they are tiny and shared by all CTAs.
+//    ahead of use in ping-pong registers; they are tiny and shared by all CTAs.
 //  * Weights are decoded with Blackwell's native converts: one
 //    cvt.rn.f16x2.e2m1x2 per two FP4 codes (exact), the UE4M3 block scale
 //    with cvt.rn.f16x2.e4m3x2 and one f16x2 multiply (exact: e2m1 * ue4m3 has
@@ -62,13 +64,33 @@ namespace skinny {
 // each later stage is issued by the warp that is last to release the ring
 // slot it refills.
 #ifndef SKINNY_STRIPS_PER_WARP
-#define SKINNY_STRIPS_PER_WARP 2
+#define SKINNY_STRIPS_PER_WARP 4
 #endif
-constexpr int kStripsPerWarp = SKINNY_STRIPS_PER_WARP;          // 2: 16 warps, 4: 8 warps
+constexpr int kStripsPerWarp = SKINNY_STRIPS_PER_WARP;          // 4: 8 consumer warps, 2: 16
 constexpr int kStripGroups = kStrips / kStripsPerWarp;
 constexpr int kChunkPairs = kChunks / 2;                        // 4
 constexpr int kConsumerWarps = kStripGroups * kChunkPairs;
-constexpr int kThreads = kConsumerWarps * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+// With a producer warpgroup (4 warps after the consumers) one thread of it
+// refills the ring slots; the consumers only wait, compute and release.  The
+// warpgroup hands its registers to the consumers (setmaxnreg).
+#ifndef SKINNY_PRODUCER
+#define SKINNY_PRODUCER 1
+#endif
+constexpr bool kProducer = SKINNY_PRODUCER != 0;
+constexpr int kProducerWarps = kProducer ? 4 : 0;
+constexpr int kThreads = kConsumerThreads + kProducerWarps * 32;
+// Registers per thread: at launch (65536 / kThreads, rounded down to 8), then
+// after the warpgroups re-balance (producer 24, consumers the rest).
+constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
+constexpr int kProducerRegs = 24;
+constexpr int kConsumerRegs = kProducer ? ((kLaunchRegs * kThreads - kProducerRegs * kProducerWarps * 32) /
+                                           kConsumerThreads) / 8 * 8 > 240 ? 240 :
+                                          ((kLaunchRegs * kThreads - kProducerRegs * kProducerWarps * 32) /
+                                           kConsumerThreads) / 8 * 8
+                                        : kLaunchRegs;
+static_assert(!kProducer || kConsumerRegs * kConsumerThreads + kProducerRegs * kProducerWarps * 32 <=
+                                kLaunchRegs * kThreads, "register split exceeds the launch total");
 // (strip, row half) pairs of a strip group finished by each of its warps.
 constexpr int kFinishPerWarp = kStripsPerWarp / 2;
 static_assert(kStripsPerWarp == 2 || kStripsPerWarp == 4, "2 or 4 strips per warp");
@@ -346,7 +368,7 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[kFinishPerWa
     float* act = reinterpret_cast<float*>(smem + Smem<FMT, NB>::kActOff);   // [128 rows][kTok tokens]
     const int gid = lane >> 2, t = lane & 3;
     const Member& mb = p.mem[0];   // the fused SiLU*mul runs one GEMM per launch
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);   // earlier readers of act are done
+    ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);   // earlier readers of act are done
 #pragma unroll
     for (int f = 0; f < kFinishPerWarp; ++f) {
         const int r = finish_strip(sg, kq, f) * kStripRows + gid + 8 * finish_half(kq, f);
@@ -356,12 +378,12 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[kFinishPerWa
             act[r * kTok + kBlockTokens * nb + 2 * t + 1] = v[f][nb][1] * mb.out_scale;
         }
     }
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
-    const int jl = threadIdx.x % 64;                     // 64 outputs x kThreads/64 tokens per pass
+    ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);
+    const int jl = threadIdx.x % 64;                     // 64 outputs x kConsumerThreads/64 tokens per pass
     const int F = mb.N / 2, j = g * 64 + jl;
 #pragma unroll
-    for (int pass = 0; pass < kTok / (kThreads / 64); ++pass) {
-        const int m = threadIdx.x / 64 + (kThreads / 64) * pass;
+    for (int pass = 0; pass < kTok / (kConsumerThreads / 64); ++pass) {
+        const int m = threadIdx.x / 64 + (kConsumerThreads / 64) * pass;
         if (m < p.M && j < F) {
             const float gate = act[jl * kTok + m], up = act[(64 + jl) * kTok + m];
             const float val = gate / (1.f + expf(-gate)) * up;
@@ -453,7 +475,7 @@ __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4]
         for (int f = 0; f < F; ++f)
             load_residual<NB, GR>(p, g, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
     }
-    ptx::named_barrier_sync(kBarConsumers, kConsumerWarps * 32);
+    ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);
     float tot[F][NB][2];
 #pragma unroll
     for (int f = 0; f < F; ++f)
@@ -687,7 +709,8 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
 {
     using S = Smem<FMT, NB>;
     constexpr int kStages = S::kStages;
-    constexpr bool kAhead = NB == 1;
+    // Activations one tile ahead in ping-pong registers, where the registers allow.
+    constexpr bool kAhead = NB == 1 || kConsumerRegs >= 200;
     const int gid = lane >> 2, t = lane & 3;
     const int sg = warp % kStripGroups, kq = warp / kStripGroups;
     const int n_units = sc.n_units;
@@ -780,8 +803,10 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         if (ok) {
             w.compute(smem32 + s * S::kStageBytes, cur);
             __syncwarp();
-            if (lane == 0) {
-                // Release the slot; the last of the 16 warps to do so refills it.
+            if (kProducer) {
+                if (lane == 0) ptx::mbar_arrive(&empty[s]);   // the producer refills the slot
+            } else if (lane == 0) {
+                // Release the slot; the last of the consumer warps to do so refills it.
                 ptx::mbar_arrive(&empty[s]);
                 if (atomicAdd(&released[s], 1) == kConsumerWarps - 1) {
                     released[s] = 0;
@@ -885,6 +910,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             issue_stage<FMT, NB, GR>(p, smem, full, q, sc.u_last - q);
     }
     __syncthreads();
+    if constexpr (kProducer) {
+        if (warp >= kConsumerWarps) {
+            // The producer warpgroup: hand registers to the consumers, then
+            // one thread refills each slot once every consumer warp has
+            // released it (tiles kStages.. of the range; the first are in flight).
+            ptx::setmaxnreg_dec<kProducerRegs>();
+            if (warp == kConsumerWarps && lane == 0) {
+                for (int q = S::kStages; q < sc.n_units; ++q) {
+                    const int s = q % S::kStages;
+                    if (!ptx::mbar_wait(&empty[s], ((q / S::kStages) - 1) & 1, kWaitLimitNs)) {
+                        atomicOr(&g_device_error, kErrEmptyWait);
+                        break;
+                    }
+                    issue_stage<FMT, NB, GR>(p, smem, full, s, sc.u_last - q);
+                }
+            }
+            return;
+        }
+        ptx::setmaxnreg_inc<kConsumerRegs>();
+    }
     // x, y, the channel scales and the workspace may belong to the previous
     // kernel: touch them only once it has completed.
     ptx::pdl_wait_prior_grid();
@@ -894,14 +939,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (p.argmax) {
         // The CTA that finishes last turns the maxima into (row, value) per
         // token and leaves the keys and the counter at zero for the next call.
+        // (Barriers among the consumer warps only.)
         __shared__ int last_cta;
-        __syncthreads();   // every warp's shared-memory maxima are in
+        ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);   // every warp's shared-memory maxima are in
         if (threadIdx.x < p.M && s_argmax_best[threadIdx.x] != 0ull)
             atomicMax(&p.amax_key[threadIdx.x], s_argmax_best[threadIdx.x]);
-        __syncthreads();   // this CTA's global atomics are issued
+        ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);   // this CTA's global atomics are issued
         if (threadIdx.x == 0)
             last_cta = ptx::atomic_add_acq_rel_gpu(p.amax_done, 1) == (int)gridDim.x - 1;
-        __syncthreads();
+        ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);
         if (last_cta && threadIdx.x < p.M) {
             const unsigned long long key = ptx::ld_volatile_u64(&p.amax_key[threadIdx.x]);
             p.out_idx[threadIdx.x] = argmax_key_row(key);
@@ -924,10 +970,19 @@ struct DeviceState {
 static std::mutex g_mu;
 static DeviceState g_dev[kMaxDevices];
 
-// Raise one kernel's dynamic shared-memory limit to what it uses; true on failure.
+// Raise one kernel's dynamic shared-memory limit to what it uses; true on
+// failure.  With a producer warpgroup, the kernel must also be launched with
+// exactly the registers per thread that its warpgroups re-balance (the
+// consumers' setmaxnreg.inc would otherwise wait for registers that never
+// come): a build that does not match is refused here, before any launch.
 template <int FMT, int NB, bool GR>
 static bool set_smem()
 {
+    if (kProducer) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, gemm_kernel<FMT, NB, GR>) != cudaSuccess || fa.numRegs != kLaunchRegs)
+            return true;
+    }
     return cudaFuncSetAttribute(gemm_kernel<FMT, NB, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Smem<FMT, NB>::kBytes) != cudaSuccess;
 }
