@@ -151,8 +151,8 @@ struct Tile<SKINNY_FMT_FP8> {
 };
 
 // Shared memory: kStages ring stages (one tile each), then the flush exchange
-// buffer (two parities of 16 warps x 2 strips x NB token blocks x 32 lanes x
-// float4), then the mbarriers and the per-slot release counters, then (NVFP4)
+// buffer (two parities of kConsumerWarps x kStripsPerWarp strips x NB token
+// blocks x 32 lanes x float4), then the mbarriers and the per-slot release counters, then (NVFP4)
 // the buffer of the fused SiLU*mul epilogue.  With two token blocks the FP8
 // ring has two slots (three do not fit next to the doubled exchange buffer).
 template <int FMT, int NB>
@@ -192,7 +192,7 @@ struct Member {
 struct Params {
     Member mem[SKINNY_MAX_GROUP];
     int n_members;
-    uint2* partials;              // [P][16 warps][32 lanes][NB] encoded float pairs (split-K only)
+    uint2* partials;              // [P][consumer warps][32 lanes][kFinishPerWarp * NB] encoded float pairs (split K)
     int M, K;
     int C;                        // K tiles per row tile
     int U;                        // tiles in total (G * C)
@@ -632,11 +632,14 @@ struct Consumer {
                 for (int r = 0; r < 4; ++r) tot[q][nb][r] = acc[0][q][nb][r] + acc[1][q][nb][r];
     }
 
-    // The warp's four strip chunks of the tile at shared address `tile`;
+    // The warp's strip chunks of the tile at shared address `tile`;
     // bx[u][nb] holds the activations of chunk 2kq + u for token block nb.
     // All shared loads are issued first, then the decode and MMA steps of the
     // chains interleave; each decoded fragment feeds one MMA per token block.
-    __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][NB][8])
+    // NVFP4 calls `mid` half-way through the MMAs (the caller loads the next
+    // tile's activations there).
+    template <class Mid>
+    __device__ __forceinline__ void compute(uint32_t tile, const uint32_t (&bx)[2][NB][8], Mid&& mid)
     {
         if constexpr (FMT == SKINNY_FMT_NVFP4) {
             uint4 cw[2][Q];
@@ -656,7 +659,8 @@ struct Consumer {
                     s8[u][q] = ptx::dup_hi(sc);   // scale of row gid+8
                 }
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 4; ++j) {
+                if (j == 2) mid();
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -670,6 +674,7 @@ struct Consumer {
                         for (int nb = 0; nb < NB; ++nb)
                             ptx::mma_f16_16816(acc[u][q][nb], a, bx[u][nb][2 * j], bx[u][nb][2 * j + 1]);
                     }
+            }
         } else {
             uint4 cw[2][Q][2];
 #pragma unroll
@@ -699,10 +704,11 @@ struct Consumer {
     }
 };
 
-// The consumer loop of one warp over the CTA's range of tiles.  With one
-// token block the activations of the next tile are fetched one tile ahead
-// into ping-pong registers; with two there is no room for a second set, and
-// each tile's activations are fetched as the tile begins (before its wait).
+// The consumer loop of one warp over the CTA's range of tiles.  The
+// activations of the next tile are fetched one tile ahead into ping-pong
+// registers where the registers allow (always with the producer warpgroup's
+// registers); otherwise each tile's activations are fetched as the tile
+// begins (before its wait) and the next tile's lines are pulled into L1.
 template <int FMT, int NB, bool GR>
 __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, const Sched& sc, int warp,
                         int lane)
@@ -789,7 +795,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     uint32_t phase = 0;
     // One tile: wait for its slot, flush the previous row tile if this one
     // starts a new one, decode and multiply, release the slot.
-    auto body = [&](int i, const uint32_t (&cur)[2][NB][8]) {
+    auto body = [&](int i, const uint32_t (&cur)[2][NB][8], auto&& mid) {
         if (ok) {
             // All lanes agree on the outcome, so the warp stays converged.
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[s], phase, kWaitLimitNs));
@@ -801,7 +807,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
             cur_g = g;
         }
         if (ok) {
-            w.compute(smem32 + s * S::kStageBytes, cur);
+            w.compute(smem32 + s * S::kStageBytes, cur, mid);
             __syncwarp();
             if (kProducer) {
                 if (lane == 0) ptx::mbar_arrive(&empty[s]);   // the producer refills the slot
@@ -834,10 +840,20 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         uint32_t bx[2][2][NB][8];   // ping-pong: [buffer][chunk][token block][words]
         fetch(bx[0]);
         // The loop is unrolled by two so the ping-pong buffers stay in registers.
+        // An MMA reads its register operands when it executes, so loading
+        // into `nxt` right after the previous tile's MMAs were issued stalls
+        // until they have.  NVFP4 loads half-way through this tile's MMAs
+        // instead (measured faster); FP8 loads before the tile.
         auto step = [&](int i, uint32_t (&cur)[2][NB][8], uint32_t (&nxt)[2][NB][8]) {
             advance();
-            if (i + 1 < n_units) fetch(nxt);   // next tile's activations, one tile ahead
-            body(i, cur);
+            if constexpr (FMT == SKINNY_FMT_NVFP4) {
+                body(i, cur, [&] {
+                    if (i + 1 < n_units) fetch(nxt);
+                });
+            } else {
+                if (i + 1 < n_units) fetch(nxt);   // next tile's activations, one tile ahead
+                body(i, cur, [] {});
+            }
         };
         int i = 0;
         for (; i + 1 < n_units; i += 2) {
@@ -854,7 +870,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
             fetch(bx);
             advance();
             if (i + 1 < n_units) prefetch_l1();
-            body(i, bx);
+            body(i, bx, [] {});
         }
     }
 
