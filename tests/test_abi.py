@@ -210,3 +210,16 @@ def test_grouped_rejects_bad_m_k_and_dtype():
     assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 520, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
     assert lib.skinny_nvfp4_gemm_grouped(arr, 2, 1, 512, 3, None, 0, None) == sk.ERR_INVALID_ARG
     assert lib.skinny_nvfp4_gemm_grouped(None, 2, 1, 512, sk.OUT_F32, None, 0, None) == sk.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("buf, nbytes, method, status", [
+    (None, 1 << 20, 0, "SKINNY_ERR_INVALID_ARG"),        # no buffer
+    (ALIGNED, 8, 0, "SKINNY_ERR_INVALID_ARG"),           # fewer than 16 bytes
+    (ALIGNED, 1 << 20, 2, "SKINNY_ERR_INVALID_ARG"),     # no such method
+    (ALIGNED + 4, 1 << 20, 1, "SKINNY_ERR_ALIGNMENT"),   # not 16-byte aligned
+])
+def test_stream_read_argument_checks(buf, nbytes, method, status):
+    """The read-only ceiling kernels validate their arguments before any CUDA call."""
+    lib = sk.library()
+    st = lib.skinny_stream_read(buf, nbytes, method, None, None)
+    assert sk.status_string(st) == status
