@@ -93,6 +93,11 @@ static_assert(!kProducer || kConsumerRegs * kConsumerThreads + kProducerRegs * k
                                 kLaunchRegs * kThreads, "register split exceeds the launch total");
 // (strip, row half) pairs of a strip group finished by each of its warps.
 constexpr int kFinishPerWarp = kStripsPerWarp / 2;
+// With the producer warpgroup, an NVFP4 ring slot is released by every lane
+// of the consumer warps (empty barrier count kConsumerThreads); FP8 releases
+// once per warp after a warp barrier (measured faster each way).
+template <int FMT>
+constexpr bool kLaneRelease = FMT == SKINNY_FMT_NVFP4;
 static_assert(kStripsPerWarp == 2 || kStripsPerWarp == 4, "2 or 4 strips per warp");
 
 // The f-th (strip, row half) pair that warp (sg, kq) finishes: strip
@@ -808,19 +813,25 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         }
         if (ok) {
             w.compute(smem32 + s * S::kStageBytes, cur, mid);
-            __syncwarp();
-            if (kProducer) {
-                if (lane == 0) ptx::mbar_arrive(&empty[s]);   // the producer refills the slot
-            } else if (lane == 0) {
-                // Release the slot; the last of the consumer warps to do so refills it.
+            if (kProducer && kLaneRelease<FMT>) {
+                // Every lane releases its own reads of the slot: no warp
+                // barrier before the release (measured faster for NVFP4).
                 ptx::mbar_arrive(&empty[s]);
-                if (atomicAdd(&released[s], 1) == kConsumerWarps - 1) {
-                    released[s] = 0;
-                    if (i + kStages < n_units) {
-                        if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
-                            issue_stage<FMT, NB, GR>(p, smem, full, s, sc.u_last - (i + kStages));
-                        else
-                            atomicOr(&g_device_error, kErrEmptyWait);
+            } else {
+                __syncwarp();
+                if (kProducer) {
+                    if (lane == 0) ptx::mbar_arrive(&empty[s]);   // the producer refills the slot
+                } else if (lane == 0) {
+                    // Release the slot; the last of the consumer warps to do so refills it.
+                    ptx::mbar_arrive(&empty[s]);
+                    if (atomicAdd(&released[s], 1) == kConsumerWarps - 1) {
+                        released[s] = 0;
+                        if (i + kStages < n_units) {
+                            if (ptx::mbar_wait(&empty[s], phase, kWaitLimitNs))
+                                issue_stage<FMT, NB, GR>(p, smem, full, s, sc.u_last - (i + kStages));
+                            else
+                                atomicOr(&g_device_error, kErrEmptyWait);
+                        }
                     }
                 }
             }
@@ -916,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         ptx::pdl_launch_dependents();
         for (int s = 0; s < S::kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], kConsumerWarps);
+            ptx::mbar_init(&empty[s], kLaneRelease<FMT> && kProducer ? kConsumerThreads : kConsumerWarps);
             reinterpret_cast<int*>(smem + S::kCountOff)[s] = 0;
         }
         ptx::fence_mbar_init();
