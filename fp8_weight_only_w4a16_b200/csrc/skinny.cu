@@ -56,13 +56,13 @@
 
 namespace skinny {
 
-// All warps are consumers.  A warp handles kStripsPerWarp consecutive strips
-// (strip group sg = w % kStripGroups) and the chunk pair kq = w / kStripGroups
-// (chunks 2kq, 2kq+1) of every tile, so the kChunkPairs warps of a strip
-// group hold the four K quarters of the same rows and add them at flush
-// time.  There is no producer warp: thread 0 issues the first stages, and
-// each later stage is issued by the warp that is last to release the ring
-// slot it refills.
+// Consumer warp w handles kStripsPerWarp consecutive strips (strip group
+// sg = w % kStripGroups) and the chunk pair kq = w / kStripGroups (chunks
+// 2kq, 2kq+1) of every tile, so the kChunkPairs warps of a strip group hold
+// the four K quarters of the same rows and add them at flush time.  Thread 0
+// issues the first ring stages; the later ones are issued by a producer
+// warpgroup (below), or, built without it, by the consumer warp that is last
+// to release the ring slot it refills.
 #ifndef SKINNY_STRIPS_PER_WARP
 #define SKINNY_STRIPS_PER_WARP 4
 #endif
@@ -112,7 +112,7 @@ constexpr int kMaxDevices = 64;
 
 
 
-// Named barrier id of the 16 consumer warps (0 is __syncthreads).
+// Named barrier id of the consumer warps (0 is __syncthreads).
 constexpr uint32_t kBarConsumers = 1;
 
 // Bits of g_device_error: which bounded wait gave up.
@@ -361,7 +361,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], c
     }
 }
 
-// Fused SiLU*mul epilogue of row tile g (all 16 warps of the CTA): rows
+// Fused SiLU*mul epilogue of row tile g (all consumer warps of the CTA): rows
 // 0..63 of the tile are gate rows 64g.., rows 64..127 the matching up rows,
 // so the tile yields outputs j = 64g + 0..63 of every token:
 // y[m][j] = silu(gate) * up, silu(z) = z / (1 + e^-z), in FP32.
@@ -1038,7 +1038,8 @@ static int current_device(int* sms)
 
 // Workspace layout (identical for every shape and M on a device, so one
 // workspace can serve calls of different shapes in turn): one partial-sum slot
-// of 16 warps x 32 lanes x 2 token blocks x 2 floats (8 KB) per CTA, for up to
+// of 8 consumer warps x 32 lanes x kFinishPerWarp pairs x 2 token blocks x 2
+// floats (8 KB) per CTA, for up to
 // one CTA per SM, then the fused argmax's running maxima (one 64-bit key per
 // token) and CTA counter.
 constexpr size_t kArgmaxTailBytes = 256;
