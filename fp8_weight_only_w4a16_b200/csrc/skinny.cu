@@ -121,6 +121,16 @@ constexpr unsigned kErrEmptyWait = 2u;     // the refilling warp waiting for a s
 constexpr unsigned kErrDrainWait = 4u;     // draining copies in flight after an abort
 constexpr unsigned kErrPartialWait = 8u;   // a finisher waiting for a partial sum
 
+// What the finished outputs of a row tile turn into.  Each kind is its own
+// kernel instance, so a launch carries only its own epilogue's code: the
+// runtime switch between them cost the plain GEMMs 3-10%.
+enum : int {
+    kEpStore = 0,     // y = scale * acc
+    kEpAdd = 1,       // y = scale * acc + residual
+    kEpSiluMul = 2,   // y = silu(gate) * up (NVFP4, gate+up packing, one GEMM)
+    kEpArgmax = 3,    // per-token (row, value) of the maximum (NVFP4, one GEMM)
+};
+
 __device__ unsigned int g_device_error;
 
 // Fused argmax: this CTA's best key per token, folded into the global maxima
@@ -323,7 +333,7 @@ __device__ __forceinline__ int argmax_key_row(unsigned long long key) { return (
 // all 32 lanes.  With the fused argmax the outputs only update this lane's
 // running best keys (best[0], best[1]); they are reduced across the CTA once,
 // at the end of the kernel.
-template <int FMT, bool GR>
+template <int FMT, bool GR, int EP>
 __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], const float (&res)[2], int g,
                                          int strip, int h, int lane, int tok0, unsigned long long (&best)[2])
 {
@@ -331,7 +341,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], c
     const Member& mb = p.mem[member_of_row<GR>(p, g)];
     const int n = (g - mb.g_begin) * kTileRows + strip * kStripRows + gid + 8 * h;
     const float sc = (FMT == SKINNY_FMT_NVFP4) ? mb.out_scale : (n < mb.N ? mb.channel_scale[n] : 0.f);
-    if (p.argmax) {
+    if constexpr (EP == kEpArgmax) {
         // The value is the one the FP32-output GEMM would store.
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -353,7 +363,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const float (&v)[2], c
         // Fused residual add: one FP32 add, then the single output rounding.
         // Each element is read (early, by load_residual) and written by this
         // thread only, so the residual may be y itself.
-        if (mb.residual) val = __fadd_rn(val, res[e]);
+        if constexpr (EP == kEpAdd) val = __fadd_rn(val, res[e]);
         if (p.out_f32)
             static_cast<float*>(mb.y)[idx] = val;
         else
@@ -429,19 +439,19 @@ __device__ __forceinline__ void load_residual(const Params& p, int g, int strip,
 // The finished outputs of row tile g (this warp's slice) go to y, to the
 // fused argmax, or through the fused SiLU*mul.  Called by every warp of the
 // CTA together.
-template <int FMT, int NB, bool GR>
+template <int FMT, int NB, bool GR, int EP>
 __device__ __forceinline__ void finish(const Params& p, const float (&v)[kFinishPerWarp][NB][2],
                                        const float (&res)[kFinishPerWarp][NB][2], int g, int sg, int kq, int lane,
                                        uint8_t* smem, unsigned long long (&best)[NB][2])
 {
-    if (FMT == SKINNY_FMT_NVFP4 && !GR && p.silu_mul) {
+    if constexpr (EP == kEpSiluMul) {
         silu_mul_epilogue<FMT, NB>(p, v, g, sg, kq, lane, smem);
     } else {
 #pragma unroll
         for (int f = 0; f < kFinishPerWarp; ++f)
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb)
-                epilogue<FMT, GR>(p, v[f][nb], res[f][nb], g, finish_strip(sg, kq, f), finish_half(kq, f), lane,
+                epilogue<FMT, GR, EP>(p, v[f][nb], res[f][nb], g, finish_strip(sg, kq, f), finish_half(kq, f), lane,
                                   kBlockTokens * nb, best[nb]);
     }
 }
@@ -460,7 +470,7 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[kFinish
 // Which case applies is the same for every warp of the CTA, so the barriers
 // of the exchange and of the fused epilogues are reached by all of them.
 // With two token blocks every lane carries both blocks' sums (NB pairs).
-template <int FMT, int NB, bool GR>
+template <int FMT, int NB, bool GR, int EP>
 __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4], int g, int c_first, int c_last,
                       int parity, uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2])
 {
@@ -475,7 +485,7 @@ __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4]
             xchg[((warp * kStripsPerWarp + q) * NB + nb) * 32 + lane] =
                 make_float4(acc[q][nb][0], acc[q][nb][1], acc[q][nb][2], acc[q][nb][3]);
     float res[F][NB][2];
-    if (c_first == c_last || b == c_last) {
+    if (EP == kEpAdd && (c_first == c_last || b == c_last)) {
 #pragma unroll
         for (int f = 0; f < F; ++f)
             load_residual<NB, GR>(p, g, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
@@ -499,7 +509,7 @@ __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4]
                 tot[f][nb][1] += hi ? v.w : v.y;
             }
     if (c_first == c_last) {
-        finish<FMT, NB, GR>(p, tot, res, g, sg, kq, lane, smem, best);
+        finish<FMT, NB, GR, EP>(p, tot, res, g, sg, kq, lane, smem, best);
         return;
     }
     constexpr int kSlot = F * NB;   // uint2 per lane
@@ -571,7 +581,7 @@ __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4]
             sum[f][nb][0] += tot[f][nb][0];
             sum[f][nb][1] += tot[f][nb][1];
         }
-    finish<FMT, NB, GR>(p, sum, res, g, sg, kq, lane, smem, best);
+    finish<FMT, NB, GR, EP>(p, sum, res, g, sg, kq, lane, smem, best);
 }
 
 // Put tile `u` into ring slot s with one bulk copy.
@@ -714,7 +724,7 @@ struct Consumer {
 // registers where the registers allow (always with the producer warpgroup's
 // registers); otherwise each tile's activations are fetched as the tile
 // begins (before its wait) and the next tile's lines are pulled into L1.
-template <int FMT, int NB, bool GR>
+template <int FMT, int NB, bool GR, int EP>
 __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, const Sched& sc, int warp,
                         int lane)
 {
@@ -766,7 +776,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         w.total(tot);
         const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
         const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
-        flush<FMT, NB, GR>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane, best);
+        flush<FMT, NB, GR, EP>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane, best);
         parity ^= 1;
     };
     auto fetch = [&](uint32_t (&dst)[2][NB][8]) {
@@ -886,7 +896,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
 
     if (n_units > 0) flush_g(cur_g);
-    if (p.argmax) {
+    if constexpr (EP == kEpArgmax) {
         // The lanes with the same t hold the same tokens for different rows:
         // reduce over them, then one shared-memory atomic per token per warp.
 #pragma unroll
@@ -911,7 +921,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
     }
 }
 
-template <int FMT, int NB, bool GR>
+template <int FMT, int NB, bool GR, int EP>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p)
 {
     using S = Smem<FMT, NB>;
@@ -961,9 +971,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // kernel: touch them only once it has completed.
     ptx::pdl_wait_prior_grid();
 
-    consume<FMT, NB, GR>(p, smem, full, empty, sc, warp, lane);
+    consume<FMT, NB, GR, EP>(p, smem, full, empty, sc, warp, lane);
 
-    if (p.argmax) {
+    if constexpr (EP == kEpArgmax) {
         // The CTA that finishes last turns the maxima into (row, value) per
         // token and leaves the keys and the counter at zero for the next call.
         // (Barriers among the consumer warps only.)
@@ -1002,16 +1012,27 @@ static DeviceState g_dev[kMaxDevices];
 // exactly the registers per thread that its warpgroups re-balance (the
 // consumers' setmaxnreg.inc would otherwise wait for registers that never
 // come): a build that does not match is refused here, before any launch.
-template <int FMT, int NB, bool GR>
+template <int FMT, int NB, bool GR, int EP>
 static bool set_smem()
 {
     if (kProducer) {
         cudaFuncAttributes fa{};
-        if (cudaFuncGetAttributes(&fa, gemm_kernel<FMT, NB, GR>) != cudaSuccess || fa.numRegs != kLaunchRegs)
+        if (cudaFuncGetAttributes(&fa, gemm_kernel<FMT, NB, GR, EP>) != cudaSuccess || fa.numRegs != kLaunchRegs)
             return true;
     }
-    return cudaFuncSetAttribute(gemm_kernel<FMT, NB, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(gemm_kernel<FMT, NB, GR, EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Smem<FMT, NB>::kBytes) != cudaSuccess;
+}
+
+// Every instance a launch of this format and token-block count can pick.
+template <int FMT, int NB>
+static bool set_smem_nb()
+{
+    if (set_smem<FMT, NB, false, kEpStore>() || set_smem<FMT, NB, false, kEpAdd>()) return true;
+    if constexpr (FMT == SKINNY_FMT_NVFP4)
+        return set_smem<FMT, NB, false, kEpSiluMul>() || set_smem<FMT, NB, false, kEpArgmax>() ||
+               set_smem<FMT, NB, true, kEpStore>();
+    return false;
 }
 
 // SM count of the current device; sets the kernels' shared-memory limit once.
@@ -1025,9 +1046,8 @@ static int current_device(int* sms)
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             return SKINNY_ERR_CUDA;
-        if (set_smem<SKINNY_FMT_NVFP4, 1, false>() || set_smem<SKINNY_FMT_NVFP4, 2, false>() ||
-            set_smem<SKINNY_FMT_NVFP4, 1, true>() || set_smem<SKINNY_FMT_NVFP4, 2, true>() ||
-            set_smem<SKINNY_FMT_FP8, 1, false>() || set_smem<SKINNY_FMT_FP8, 2, false>())
+        if (set_smem_nb<SKINNY_FMT_NVFP4, 1>() || set_smem_nb<SKINNY_FMT_NVFP4, 2>() ||
+            set_smem_nb<SKINNY_FMT_FP8, 1>() || set_smem_nb<SKINNY_FMT_FP8, 2>())
             return SKINNY_ERR_CUDA;
         d.sms = n;
         d.ready = true;
@@ -1100,6 +1120,20 @@ static Params single(const void* x, int M, int64_t K, const void* w_packed, cons
     return p;
 }
 
+// The kernel instance for NB token blocks and epilogue kind ep (grouped
+// launches store their outputs).
+template <int FMT, int NB>
+static cudaError_t launch_instance(const cudaLaunchConfig_t& cfg, const Params& p, int ep)
+{
+    if constexpr (FMT == SKINNY_FMT_NVFP4) {
+        if (p.n_members > 1) return cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, NB, true, kEpStore>, p);
+        if (ep == kEpSiluMul) return cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, NB, false, kEpSiluMul>, p);
+        if (ep == kEpArgmax) return cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, NB, false, kEpArgmax>, p);
+    }
+    if (ep == kEpAdd) return cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, NB, false, kEpAdd>, p);
+    return cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, NB, false, kEpStore>, p);
+}
+
 // Launch the GEMM(s) of p, whose members' row tiles add up to G.
 template <int FMT>
 static int launch(Params p, int64_t G, int64_t K, void* workspace, size_t workspace_bytes, cudaStream_t stream)
@@ -1135,16 +1169,10 @@ static int launch(Params p, int64_t G, int64_t K, void* workspace, size_t worksp
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    if constexpr (FMT == SKINNY_FMT_NVFP4) {
-        if (p.n_members > 1)
-            e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, true> : gemm_kernel<FMT, 1, true>, p);
-        else
-            e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, false> : gemm_kernel<FMT, 1, false>, p);
-    } else {
-        if (p.n_members != 1) return SKINNY_ERR_UNSUPPORTED;
-        e = cudaLaunchKernelEx(&cfg, two_blocks ? gemm_kernel<FMT, 2, false> : gemm_kernel<FMT, 1, false>, p);
-    }
+    if (FMT != SKINNY_FMT_NVFP4 && (p.n_members != 1 || p.argmax || p.silu_mul)) return SKINNY_ERR_UNSUPPORTED;
+    if (p.n_members > 1 && (p.argmax || p.silu_mul)) return SKINNY_ERR_UNSUPPORTED;
+    const int ep = p.argmax ? kEpArgmax : p.silu_mul ? kEpSiluMul : p.mem[0].residual ? kEpAdd : kEpStore;
+    const cudaError_t e = two_blocks ? launch_instance<FMT, 2>(cfg, p, ep) : launch_instance<FMT, 1>(cfg, p, ep);
     if (e != cudaSuccess) return SKINNY_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SKINNY_OK : SKINNY_ERR_CUDA;
 }
