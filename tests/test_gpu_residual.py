@@ -100,3 +100,27 @@ def test_add_equals_plain_gemm_plus_residual_in_fp32():
     sk.gemm_add_into(y, xt, w, r, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(y, y_plain + r)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "fp8"])
+@pytest.mark.parametrize("M", [12, 16])
+def test_add_with_two_token_blocks(fmt, M):
+    """The residual-add kernels for 9 <= M <= 16 (two MMA token blocks), FP16
+    in place, split K, ragged N and K."""
+    N, K = 700, 1040
+    x = si.activations(M, K, seed=M, cfg_id=66)
+    r = residual_like(M, N, torch.float16, 30 + M)
+    if fmt == "nvfp4":
+        codes, scales = si.nvfp4_weights(N, K, seed=M, cfg_id=66)
+        w = sk.PackedNVFP4.from_logical(codes, scales, 0.5, DEV)
+        yr, b = oracle_nvfp4(x, codes, scales, 0.5)
+        ws = sk.make_workspace(sk.FMT_NVFP4, M, N, K, DEV)
+    else:
+        q, s = si.fp8_weights(N, K, seed=M, cfg_id=66)
+        w = sk.PackedFP8.from_logical(q, s, DEV)
+        yr, b = oracle_fp8(x, q, s)
+        ws = sk.make_workspace(sk.FMT_FP8, M, N, K, DEV)
+    y = torch.from_numpy(r.copy()).to(DEV)
+    sk.gemm_add_into(y, torch.from_numpy(x).to(DEV), w, y, workspace=ws)
+    torch.cuda.synchronize()
+    check(y.double().cpu().numpy(), yr + r.astype(np.float64), b, torch.float16, "%s add M=%d" % (fmt, M))
