@@ -125,6 +125,12 @@ constexpr unsigned kErrPartialWait = 8u;   // a finisher waiting for a partial s
 // What the finished outputs of a row tile turn into.  Each kind is its own
 // kernel instance, so a launch carries only its own epilogue's code: the
 // runtime switch between them cost the plain GEMMs 3-10%.
+// The FP8 kernels, which wait on HBM, load a fused add's residual as they
+// begin a row tile; the issue-bound NVFP4 kernels load it in the flush
+// (each measured faster than the other way).
+template <int FMT>
+constexpr bool kEarlyResidual = FMT == SKINNY_FMT_FP8;
+
 enum : int {
     kEpStore = 0,     // y = scale * acc
     kEpAdd = 1,       // y = scale * acc + residual
@@ -413,9 +419,9 @@ __device__ void silu_mul_epilogue(const Params& p, const float (&v)[kFinishPerWa
 }
 
 // The residual of this lane's outputs of row tile g (strip `strip`, rows
-// gid + 8h, tokens 8nb + 2t + e), loaded as soon as the CTA knows that it
-// finishes the row tile, so that the loads overlap the exchange and the
-// split-K wait instead of stalling the epilogue.  Zero where there is none.
+// gid + 8h, tokens 8nb + 2t + e), loaded ahead of the epilogue: by the FP8
+// kernels when the CTA begins a row tile it finishes, by the NVFP4 kernels in
+// the flush, before its barrier.  Zero where there is none.
 template <int NB, bool GR>
 __device__ __forceinline__ void load_residual(const Params& p, int g, int strip, int h, int lane,
                                               float (&res)[NB][2])
@@ -473,7 +479,8 @@ __device__ __forceinline__ void finish(const Params& p, const float (&v)[kFinish
 // With two token blocks every lane carries both blocks' sums (NB pairs).
 template <int FMT, int NB, bool GR, int EP>
 __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4], int g, int c_first, int c_last,
-                      int parity, uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2])
+                      int parity, uint8_t* smem, int b, int warp, int lane, unsigned long long (&best)[NB][2],
+                      const float (&res_early)[kFinishPerWarp][NB][2])
 {
     using S = Smem<FMT, NB>;
     constexpr int F = kFinishPerWarp;
@@ -486,10 +493,17 @@ __device__ void flush(const Params& p, const float (&acc)[kStripsPerWarp][NB][4]
             xchg[((warp * kStripsPerWarp + q) * NB + nb) * 32 + lane] =
                 make_float4(acc[q][nb][0], acc[q][nb][1], acc[q][nb][2], acc[q][nb][3]);
     float res[F][NB][2];
-    if (EP == kEpAdd && (c_first == c_last || b == c_last)) {
+    if constexpr (EP == kEpAdd) {
+        if constexpr (kEarlyResidual<FMT>) {
 #pragma unroll
-        for (int f = 0; f < F; ++f)
-            load_residual<NB, GR>(p, g, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
+            for (int f = 0; f < F; ++f)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) res[f][nb][0] = res_early[f][nb][0], res[f][nb][1] = res_early[f][nb][1];
+        } else if (c_first == c_last || b == c_last) {
+#pragma unroll
+            for (int f = 0; f < F; ++f)
+                load_residual<NB, GR>(p, g, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
+        }
     }
     ptx::named_barrier_sync(kBarConsumers, kConsumerThreads);
     float tot[F][NB][2];
@@ -772,12 +786,28 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) best[nb][0] = best[nb][1] = 0ull;
     // Contributors of a row tile: only the two at the ends of the range are shared.
+    // Fused residual add (FP8): the residual of a row tile this CTA finishes
+    // is loaded as the CTA begins the row tile, so the loads are long done
+    // when the epilogue needs them.  NVFP4 loads it in the flush instead.
+    float res[kFinishPerWarp][NB][2];
+    auto load_res = [&](int rg) {
+        if constexpr (EP == kEpAdd && kEarlyResidual<FMT>) {
+            const int c_first = rg == sc.first_g ? sc.first_owner : sc.b;
+            const int c_last = rg == sc.last_g ? sc.last_owner : sc.b;
+            if (c_first == c_last || sc.b == c_last) {
+                const int sg = warp % kStripGroups, kq = warp / kStripGroups;
+#pragma unroll
+                for (int f = 0; f < kFinishPerWarp; ++f)
+                    load_residual<NB, GR>(p, rg, finish_strip(sg, kq, f), finish_half(kq, f), lane, res[f]);
+            }
+        }
+    };
     auto flush_g = [&](int fg) {
         float tot[kStripsPerWarp][NB][4];
         w.total(tot);
         const int c_first = fg == sc.first_g ? sc.first_owner : sc.b;
         const int c_last = fg == sc.last_g ? sc.last_owner : sc.b;
-        flush<FMT, NB, GR, EP>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane, best);
+        flush<FMT, NB, GR, EP>(p, tot, fg, c_first, c_last, parity, smem, sc.b, warp, lane, best, res);
         parity ^= 1;
     };
     auto fetch = [&](uint32_t (&dst)[2][NB][8]) {
@@ -815,6 +845,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
             flush_g(cur_g);
             w.zero();
             cur_g = g;
+            load_res(cur_g);
         }
     };
     // One tile: wait for its slot, flush the previous row tile if this one
@@ -863,6 +894,7 @@ __device__ void consume(const Params& p, uint8_t* smem, uint64_t* full, uint64_t
         --c;
     };
 
+    if (n_units > 0) load_res(cur_g);
     if constexpr (kAhead) {
         uint32_t bx[2][2][NB][8];   // ping-pong: [buffer][chunk][token block][words]
         fetch(bx[0]);
